@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Benchmark of the W8A8 linear layer on B200.
+
+One step = one pass of the Prefill hot path over one batch at 7B shapes:
+per-token dynamic quantization of X [2048, 4096] (bf16) and the tcgen05 INT8
+GEMM against the shared per-channel INT8 weight [11008, 4096] with the
+dequant + bias epilogue fused in, bf16 output [2048, 11008]. The weight is
+quantized once before timing (load time, not part of the step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own batch
+(no collective on the data path: replicas, weak scaling); the timed region
+is bracketed by a barrier and the slowest rank's time is reported.
+--impl reference times the CPU oracle (a plain C implementation, OpenMP over
+rows) on a bounded sample of the same workload.
+
+The JSON line also carries a Decode measurement (fused static-quant linear,
+32 tokens x 4096 -> 11008, HBM-bound) under "decode".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, K, N = 2048, 4096, 11008
+DEC_M, DEC_K, DEC_N = 32, 4096, 11008
+N_SETS = 4          # rotating input/weight/output sets: 4 x ~115 MB > 126 MB L2
+METRIC = "W8A8 linear: prefill INT8 TOPS, decode HBM GB/s (fraction of B200 peak)"
+WORKLOAD = ("prefill W8A8 linear at 7B shapes: X bf16 [2048 x 4096] (row-scaled N(0,1), 6 channels x60) "
+            "-> per-token symmetric INT8 quant -> INT8 GEMM vs per-channel INT8 W [4096 x 11008] "
+            "-> fused dequant + bias -> bf16 [2048 x 11008]")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# INT8 dense tensor throughput is twice bf16 on B200 (4.5 vs 2.25 PFLOP/s nominal)
+INT8_OVER_BF16 = 2.0
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(backend: str):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def cpu_baseline_sample(rows: int, seed: int = 0):
+    """Time the oracle on `rows` tokens of the workload: per-token quant,
+    int64 GEMM and the fixed-order epilogue. Returns (seconds, ops)."""
+    import oracle
+    from int8_gemm_token_b200 import synth
+    case = synth.prefill_7b(seed)
+    Wq, s_w, _ = oracle.quant_weight_per_channel(case.W)  # load time, not timed
+    X = np.ascontiguousarray(case.X[:rows])
+    t0 = time.perf_counter()
+    Xq, S = oracle.quant_per_token(X)
+    acc = oracle.gemm_i64(Xq, Wq)
+    y = oracle.epilogue(acc, S, s_w, bias=case.bias)
+    oracle.f32_to_bf16(y)
+    dt = time.perf_counter() - t0
+    return dt, 2.0 * rows * N * K
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle, as it stands, on a bounded sample per step."""
+    if rank != 0:
+        return 0
+    import oracle
+    rows = args.ref_rows
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, ops = cpu_baseline_sample(rows, seed=0)
+        if i >= args.warmup:
+            times.append(dt)
+    per = statistics.mean(times)
+    value = 2.0 * rows * N * K / per / 1e12
+    sample = f"{rows} of {M} tokens per step (full K={K}, N={N}); value scaled to TOPS of that sample"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N},
+            "cpu_baseline": {"value": value, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    from int8_gemm_token_b200 import synth
+    from int8_gemm_token_b200 import w8a8 as W
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+
+    def bf16_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    # ---------------------------------------------------------------- data
+    sets = []
+    for i in range(N_SETS):
+        case = synth.prefill_7b(seed=1000 * rank + i)
+        X = bf16_dev(case.X)
+        Wq, s_w, cs = W.w8a8_quant_weight_per_channel(torch.from_numpy(case.W).to(dev))
+        sets.append(dict(X=X, Wq=Wq, s_w=s_w, bias=torch.from_numpy(case.bias).to(dev),
+                         Xq=torch.empty((M, K), dtype=torch.int8, device=dev),
+                         S=torch.empty((M,), dtype=torch.float32, device=dev),
+                         out=torch.empty((M, N), dtype=torch.bfloat16, device=dev)))
+        del case
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        W.w8a8_quant_per_token(s["X"], Xq=s["Xq"], S_x=s["S"], stream=stream)
+        W.w8a8_gemm_dequant(s["Xq"], s["S"], s["Wq"], s["s_w"], bias=s["bias"], out=s["out"], stream=stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for i in range(args.warmup):
+        step(sets[i % N_SETS])
+    torch.cuda.synchronize()
+
+    # ---------------------------------------------------------------- timed
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            s = sets[i % N_SETS]
+            ev[i][0].record(stream)
+            W.w8a8_quant_per_token(s["X"], Xq=s["Xq"], S_x=s["S"], stream=stream)
+            ev[i][1].record(stream)
+            W.w8a8_gemm_dequant(s["Xq"], s["S"], s["Wq"], s["s_w"], bias=s["bias"], out=s["out"], stream=stream)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    quant_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    gemm_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    ms_per_step = max_over_ranks(total_ms / args.steps)
+    ops = 2.0 * M * N * K
+    value = world * ops / (ms_per_step * 1e-3) / 1e12
+    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
+    quant_bytes = 2.0 * M * K + M * K + 4.0 * M
+    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    if W.w8a8_check_device_error() != 0:
+        raise RuntimeError("device status word set during the benchmark")
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if not args.no_e2e:
+        hostX = [sets[i]["X"].cpu().pin_memory() for i in range(N_SETS)]
+        hostOut = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(N_SETS)]
+        e2e_steps = max(3, min(args.steps, 50))
+        for i in range(3):
+            s = sets[i % N_SETS]
+            s["X"].copy_(hostX[i % N_SETS], non_blocking=True)
+            step(s)
+            hostOut[i % N_SETS].copy_(s["out"], non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            s = sets[i % N_SETS]
+            s["X"].copy_(hostX[i % N_SETS], non_blocking=True)
+            step(s)
+            hostOut[i % N_SETS].copy_(s["out"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+        e2e = {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms,
+               "steps": e2e_steps}
+
+    # ---------------------------------------------------------------- decode
+    decode = None
+    if not args.no_decode:
+        decode = bench_decode(args, dev, rank, peaks, max_over_ranks, barrier)
+
+    del sets
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            dt, sops = cpu_baseline_sample(8)
+            rows = int(min(M, max(8, 8 * args.cpu_seconds / max(dt, 1e-3))))
+            dt, sops = cpu_baseline_sample(rows)
+            cpu = {"value": sops / dt / 1e12, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                   "sample": f"{rows} of {M} tokens (full K={K}, N={N}), quant + int64 GEMM + epilogue, {dt:.1f} s"}
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "parallelism": f"replicas x{world}",
+                       "l2": f"{N_SETS} rotating X/Wq/out sets, {N_SETS * 115} MB > 126 MB L2"},
+            "roofline": {"bound": "tensor", "kernel": "gemm_i8_tc_kernel", "achieved": gemm_tops,
+                         "peak": int8_peak, "unit": "TOPS", "frac": gemm_tops / int8_peak,
+                         "peak_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (int8/bf16 nominal)",
+                         "traffic": None},
+            "quant": {"kernel": "quant_per_token_kernel", "ms": quant_ms, "achieved": quant_gbs,
+                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": quant_gbs / peaks["hbm_gbs"],
+                      "C_s_over_C_g": quant_ms / gemm_ms},
+            "gemm_ms": gemm_ms,
+            "decode": decode,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def bench_decode(args, dev, rank, peaks, max_over_ranks, barrier):
+    """Fused static-quant Decode linear, 32 x 4096 -> 11008, rotating 6 weights (> L2)."""
+    import torch
+
+    from int8_gemm_token_b200 import synth
+    from int8_gemm_token_b200 import w8a8 as W
+    n_w = 6
+    case = synth.decode_static(M=DEC_M, N=DEC_N, K=DEC_K, seed=rank)
+    X = torch.from_numpy(case.X.view(np.int16)).view(torch.bfloat16).to(dev)
+    S, r, Z = W.w8a8_calibrate_static(torch.from_numpy(case.Xcal.view(np.int16)).view(torch.bfloat16).to(dev))
+    ws = []
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(torch.from_numpy(case.W).to(dev))
+    for i in range(n_w):
+        ws.append((Wq.clone(), s_w.clone(), cs.clone(), torch.empty((DEC_M, DEC_N), dtype=torch.bfloat16, device=dev)))
+    wsz = W.w8a8_gemm_workspace_size(DEC_M, DEC_N, DEC_K)
+    work = torch.empty((max(wsz, 1),), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    steps = max(args.steps, 20)
+    for i in range(max(args.warmup, 3)):
+        q, s, c, o = ws[i % n_w]
+        W.w8a8_linear_static(X, S, r, Z, q, s, c, out=o, workspace=work, stream=stream)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier()
+    for i in range(steps):
+        q, s, c, o = ws[i % n_w]
+        ev[i][0].record(stream)
+        W.w8a8_linear_static(X, S, r, Z, q, s, c, out=o, workspace=work, stream=stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev))
+    nbytes = DEC_N * DEC_K + 8.0 * DEC_N + 2.0 * DEC_M * DEC_K + 2.0 * DEC_M * DEC_N
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": f"decode fused static-quant linear M={DEC_M} K={DEC_K} N={DEC_N}, {n_w} rotating weights",
+            "us_per_layer": ms * 1e3, "achieved": gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+            "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": nbytes}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-rows", type=int, default=16)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    if args.impl == "reference":
+        world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+        return run_reference(args, world, rank)
+    world, rank, local = dist_setup("nccl")
+    try:
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

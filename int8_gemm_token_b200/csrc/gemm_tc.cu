@@ -1,0 +1,405 @@
+// gemm_tc.cu -- INT8 x INT8 -> INT32 GEMM on the 5th-generation tensor cores
+// (tcgen05.mma kind::i8) with the dequant epilogue fused in.
+//
+// What it computes: LLM.int8() paper summary, architecture figure steps (3)
+// (INT8 matmul with INT32 accumulation) and (4) (rescale by the outer product
+// of the row and column constants), §一.2 four-term zero-point expansion
+// (with a symmetric weight only the -Z * colsum[n] term survives), and for
+// the mixed mode the 16-bit decomposition step (2) and the final sum
+// Y = X_outlier W_outlier + Dequant(Q(X_normal) Q(W_normal)).
+//
+// How (sm_100a): one persistent CTA per SM walks output tiles of 128 x BN.
+//   warp 0      TMA producer: 128-byte-swizzled K-major tiles of Xq [M, K]
+//               and Wq [N, K] into a STAGES-deep shared-memory ring;
+//   warp 1      TMEM allocator and MMA issuer: one thread issues
+//               tcgen05.mma (M=128, N=BN, K=32 bytes) into one of two TMEM
+//               accumulators (2 x BN int32 columns), tcgen05.commit frees
+//               ring slots and hands a finished accumulator to the epilogue;
+//   warps 4..7  epilogue: tcgen05.ld of the int32 accumulator (each warp its
+//               32-lane quarter), the fixed-order fp32 dequant, bf16 stores.
+// Double-buffered accumulators let the epilogue of tile i overlap the MMAs
+// of tile i+1. Every wait is bounded; on a timeout the CTA records
+// W8A8_ERR_DEVICE_TIMEOUT, stops, frees its TMEM and returns.
+#include "device.cuh"
+#include "kernels.h"
+
+namespace w8a8 {
+
+namespace {
+
+constexpr int kBM = 128;              // rows of Xq per tile = TMEM lanes
+constexpr int kBK = 128;              // bytes of K per stage = one 128B swizzle row
+constexpr int kStageA = kBM * kBK;    // 16 KiB
+constexpr int kThreads = 256;
+constexpr int kEpiWarp0 = 4;
+
+template <int BN, int STAGES>
+struct TcConfig {
+  static constexpr int kStageB = BN * kBK;
+  static constexpr int kTmemCols = 2 * BN;  // two accumulators
+  static constexpr size_t kRing = static_cast<size_t>(STAGES) * (kStageA + kStageB);
+  static constexpr size_t kSmem = kRing + 1024 /*alignment slack*/ + 256 /*barriers etc.*/;
+  static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
+};
+
+// Fixed-order epilogue of one row segment of 32 columns (see include/w8a8.h):
+//   c = acc - Z*colsum[n]; y = fmaf(float(c), S_x*s_w[n], side + bias[n]).
+template <bool MIXED>
+__device__ __forceinline__ void epilogue_chunk(const uint32_t (&acc)[32], int64_t m, int64_t n0,
+                                               int64_t M, int64_t N, float sx, int32_t z,
+                                               const EpilogueArgs &ep, int32_t nuse) {
+  if (m >= M) return;
+  const bool full = n0 + 32 <= N;
+  float sw[32], bs[32];
+  int32_t cs[32];
+  if (full) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(ep.s_w + n0) + i);
+      sw[4 * i] = v.x; sw[4 * i + 1] = v.y; sw[4 * i + 2] = v.z; sw[4 * i + 3] = v.w;
+    }
+    if (ep.bias) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(ep.bias + n0) + i);
+        bs[4 * i] = v.x; bs[4 * i + 1] = v.y; bs[4 * i + 2] = v.z; bs[4 * i + 3] = v.w;
+      }
+    }
+    if (z != 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int4 v = __ldg(reinterpret_cast<const int4 *>(ep.colsum + n0) + i);
+        cs[4 * i] = v.x; cs[4 * i + 1] = v.y; cs[4 * i + 2] = v.z; cs[4 * i + 3] = v.w;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const bool ok = n0 + i < N;
+      sw[i] = ok ? __ldg(ep.s_w + n0 + i) : 0.0f;
+      bs[i] = (ok && ep.bias) ? __ldg(ep.bias + n0 + i) : 0.0f;
+      cs[i] = (ok && z != 0) ? __ldg(ep.colsum + n0 + i) : 0;
+    }
+  }
+
+  float side[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) side[i] = 0.0f;
+  if (MIXED) {
+    for (int32_t j = 0; j < nuse; ++j) {
+      const float xo = __uint_as_float(static_cast<uint32_t>(ep.Xo[m * ep.cap + j]) << 16);
+      const uint16_t *wrow = ep.W + static_cast<int64_t>(__ldg(ep.outlier_idx + j)) * ep.ldw + n0;
+      if (full && (ep.ldw % 8) == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4 *>(wrow) + i);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            side[8 * i + 2 * h] = __fmaf_rn(xo, bf16_lo(w4[h]), side[8 * i + 2 * h]);
+            side[8 * i + 2 * h + 1] = __fmaf_rn(xo, bf16_hi(w4[h]), side[8 * i + 2 * h + 1]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (n0 + i < N) {
+            const float wv = __uint_as_float(static_cast<uint32_t>(__ldg(wrow + i)) << 16);
+            side[i] = __fmaf_rn(xo, wv, side[i]);
+          }
+        }
+      }
+    }
+  }
+
+  float y[32];
+  int32_t craw[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    int32_t c = static_cast<int32_t>(acc[i]);
+    if (z != 0) c -= z * cs[i];
+    craw[i] = c;
+    const float f = __int2float_rn(c);
+    const float sc = __fmul_rn(sx, sw[i]);
+    float add = MIXED ? side[i] : 0.0f;
+    if (ep.bias) add = __fadd_rn(add, bs[i]);
+    y[i] = __fmaf_rn(f, sc, add);
+  }
+
+  if (ep.out_dtype == W8A8_BF16) {
+    uint16_t *o = static_cast<uint16_t *>(ep.out) + m * N + n0;
+    if (full && (N % 8) == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 v;
+        v.x = pack_bf16x2(y[8 * i + 0], y[8 * i + 1]);
+        v.y = pack_bf16x2(y[8 * i + 2], y[8 * i + 3]);
+        v.z = pack_bf16x2(y[8 * i + 4], y[8 * i + 5]);
+        v.w = pack_bf16x2(y[8 * i + 6], y[8 * i + 7]);
+        reinterpret_cast<uint4 *>(o)[i] = v;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (n0 + i < N) {
+          __nv_bfloat16 b = __float2bfloat16_rn(y[i]);
+          o[i] = *reinterpret_cast<uint16_t *>(&b);
+        }
+    }
+  } else if (ep.out_dtype == W8A8_FP32) {
+    float *o = static_cast<float *>(ep.out) + m * N + n0;
+    if (full && (N % 4) == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<float4 *>(o)[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (n0 + i < N) o[i] = y[i];
+    }
+  } else {
+    int32_t *o = static_cast<int32_t *>(ep.out) + m * N + n0;
+    if (full && (N % 4) == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<int4 *>(o)[i] = make_int4(craw[4 * i], craw[4 * i + 1], craw[4 * i + 2], craw[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (n0 + i < N) o[i] = craw[i];
+    }
+  }
+}
+
+template <int BN, int STAGES, bool MIXED>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_i8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      int64_t M, int64_t N, int64_t K, const __grid_constant__ EpilogueArgs ep,
+                      int32_t *status, uint64_t limit_ns) {
+  using Cfg = TcConfig<BN, STAGES>;
+  constexpr uint32_t kIdesc = idesc_i8(kBM, BN);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = base;
+  uint8_t *sB = base + STAGES * kStageA;
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(base + Cfg::kRing);
+  uint64_t *empty_bar = full_bar + STAGES;
+  uint64_t *tfull_bar = empty_bar + STAGES;
+  uint64_t *tempty_bar = tfull_bar + 2;
+  uint64_t *drain_bar = tempty_bar + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t num_m = (M + kBM - 1) / kBM;
+  const int64_t num_n = (N + BN - 1) / BN;
+  const int64_t num_tiles = num_m * num_n;
+  const int nkb = static_cast<int>((K + kBK - 1) / kBK);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int32_t mrow = static_cast<int32_t>((tile % num_m) * kBM);
+        const int32_t nrow = static_cast<int32_t>((tile / num_m) * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag, limit_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_bar[stage], kStageA + Cfg::kStageB);
+          tma_load_2d(&tmA, &full_bar[stage], sA + stage * kStageA, kb * kBK, mrow);
+          tma_load_2d(&tmB, &full_bar[stage], sB + stage * Cfg::kStageB, kb * kBK, nrow);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+        // let the copies already issued land before the CTA's shared memory goes away
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s))
+            mbar_wait_bounded(&full_bar[s], (issued_parity >> s) & 1u, nullptr, limit_ns / 16 + 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, limit_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&full_bar[stage], phase, abort_flag, limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(sA + stage * kStageA);
+          const uint32_t b_addr = smem_addr(sB + stage * Cfg::kStageB);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k) {
+            mma_i8(d_tmem, smem_desc_k_sw128(a_addr + 32 * k), smem_desc_k_sw128(b_addr + 32 * k),
+                   kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tfull_bar[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+        mma_commit(drain_bar);  // wait for MMAs in flight before TMEM is freed
+        mbar_wait_bounded(drain_bar, 0, nullptr, limit_ns / 16 + 1);
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // -------------------------------------------------- epilogue
+    const int q = warp - kEpiWarp0;  // TMEM lane quarter of this warp (warp % 4)
+    const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
+    int32_t nuse = 0;
+    if (MIXED) nuse = min(__ldg(ep.n_out), ep.cap);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      // tcgen05.ld is warp-collective: the whole warp goes on or gives up together
+      const bool ready = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag, limit_ns));
+      if (!ready) {
+        if (lane == 0) {
+          record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const int64_t m = (tile % num_m) * kBM + q * 32 + lane;
+      const int64_t nbase = (tile / num_m) * BN;
+      float sx = 0.0f;
+      if (m < M) sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : __ldg(ep.S_x);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, r);
+        tmem_ld_wait();
+        epilogue_chunk<MIXED>(r, m, nbase + c * 32, M, N, sx, z, ep, nuse);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+template <int BN, int STAGES, bool MIXED>
+cudaError_t launch_tc_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
+                        const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
+  using Cfg = TcConfig<BN, STAGES>;
+  alignas(64) CUtensorMap tmA, tmB;
+  if (!encode_tmap_2d_u8(&tmA, Xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                         static_cast<uint64_t>(K), kBK, kBM))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d_u8(&tmB, Wq, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                         static_cast<uint64_t>(K), kBK, BN))
+    return cudaErrorInvalidValue;
+  auto kern = gemm_i8_tc_kernel<BN, STAGES, MIXED>;
+  // per function and per device; cheap enough to repeat on every launch
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(Cfg::kSmem));
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
+  const unsigned grid = static_cast<unsigned>(tiles < num_sms ? tiles : num_sms);
+  kern<<<grid, kThreads, Cfg::kSmem, s>>>(tmA, tmB, M, N, K, ep, status, kWaitLimitNs);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
+                           const EpilogueArgs &ep, bool mixed, int num_sms, int32_t *status,
+                           cudaStream_t s) {
+  if (mixed) return launch_tc_t<256, 4, true>(Xq, Wq, M, N, K, ep, num_sms, status, s);
+  return launch_tc_t<256, 4, false>(Xq, Wq, M, N, K, ep, num_sms, status, s);
+}
+
+// ---------------------------------------------------------------- self-test
+// A barrier that nothing completes: the bounded wait must give up, record
+// W8A8_ERR_DEVICE_TIMEOUT and let the kernel return.
+__global__ void wait_selftest_kernel(int32_t *status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+    if (!mbar_wait_bounded(&bar, 0, nullptr, limit_ns)) record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
+  }
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace w8a8

@@ -1,0 +1,55 @@
+// kernels.h -- launchers of libw8a8's kernels (internal; the public ABI is
+// include/w8a8.h). Every launcher returns the launch's cudaError_t.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/w8a8.h"
+
+namespace w8a8 {
+
+// Operands of the fused dequant epilogue (see w8a8_gemm_dequant and
+// int8_mixed_decomp_gemm in include/w8a8.h for the per-element formula).
+struct EpilogueArgs {
+  const float *S_x = nullptr;  // [M] or scalar
+  int32_t s_x_per_row = 1;
+  const int32_t *Z = nullptr;       // scalar or null
+  const int32_t *colsum = nullptr;  // [N], needed when Z != null
+  const float *s_w = nullptr;       // [N]
+  const float *bias = nullptr;      // [N] or null
+  // LLM.int8() side path (mixed mode only)
+  const uint16_t *Xo = nullptr;       // [M, cap] bf16
+  const int32_t *outlier_idx = nullptr;
+  const int32_t *n_out = nullptr;     // device scalar
+  int32_t cap = 0;
+  const uint16_t *W = nullptr;        // [K, N] bf16, row stride ldw
+  int64_t ldw = 0;
+  // output
+  void *out = nullptr;  // [M, N] dense
+  int32_t out_dtype = W8A8_BF16;
+};
+
+cudaError_t launch_quant_per_token(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                   int8_t *Xq, float *S_x, cudaStream_t s);
+cudaError_t launch_quant_per_tensor(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                    const float *r, const int32_t *Z, int8_t *Xq, int num_sms,
+                                    cudaStream_t s);
+cudaError_t launch_calibrate(const void *X, w8a8_dtype dt, int64_t T, int64_t K, int64_t ldx,
+                             float *S, float *r, int32_t *Z, int num_sms, cudaStream_t s);
+cudaError_t launch_quant_weight(const void *W, w8a8_dtype dt, int64_t K, int64_t N, int64_t ldw,
+                                int8_t *Wq, float *s_w, int32_t *colsum, cudaStream_t s);
+
+// tcgen05 GEMM + epilogue (prefill-sized M; any M works). mixed selects the
+// LLM.int8() side path in the epilogue.
+cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
+                           const EpilogueArgs &ep, bool mixed, int num_sms, int32_t *status,
+                           cudaStream_t s);
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_t s);
+
+// Driver entry point for tensor-map encoding (resolved once per process).
+bool encode_tmap_2d_u8(void *map, const void *base, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+
+}  // namespace w8a8

@@ -1,0 +1,316 @@
+// quant.cu -- activation and weight quantization kernels (HBM-bound).
+//
+//  * quant_per_token:  PDMIX glossary §2.3 eq. Q_prefill with Z_token = 0
+//    (configuration guide: Prefill is per-token symmetric); LLM.int8()
+//    summary §一.1 absmax equation. One fused pass: 16-byte loads of the row
+//    into registers, absmax by warp shuffles, one fp32 division per row,
+//    quantize from registers, 8-byte int8 stores.
+//  * quant_per_tensor: PDMIX glossary §2.3 eq. Q_decode (static S, Z).
+//  * calibrate_static: MinMax over all calibration elements (configuration
+//    guide Step 3: MinMax observer, asymmetric decode parameters).
+//  * quant_weight_per_channel: configuration guide Step 2 (int8 per_channel
+//    symmetric minmax weight); LLM.int8() summary step (1) C_w per column.
+#include "device.cuh"
+#include "kernels.h"
+
+namespace w8a8 {
+
+// ------------------------------------------------------------------ helpers
+// |x| of bf16 values compared on their bit patterns: for finite values the
+// magnitude bits order exactly like the magnitudes.
+__device__ __forceinline__ uint32_t absmax_bits_u4(const uint4 &v, uint32_t m) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = max(m, w[i] & 0x7FFFu);
+    m = max(m, (w[i] >> 16) & 0x7FFFu);
+  }
+  return m;
+}
+
+__device__ __forceinline__ uint2 quant8_sym(const uint4 &v, float r) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  int q[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    q[2 * i] = min(max(rne_clamped(__fmul_rn(bf16_lo(w[i]), r)), -127), 127);
+    q[2 * i + 1] = min(max(rne_clamped(__fmul_rn(bf16_hi(w[i]), r)), -127), 127);
+  }
+  return make_uint2(pack_i8x4(q[0], q[1], q[2], q[3]), pack_i8x4(q[4], q[5], q[6], q[7]));
+}
+
+__device__ __forceinline__ uint2 quant8_asym(const uint4 &v, float r, int z) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  int q[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    q[2 * i] = min(max(rne_clamped(__fmul_rn(bf16_lo(w[i]), r)) + z, -128), 127);
+    q[2 * i + 1] = min(max(rne_clamped(__fmul_rn(bf16_hi(w[i]), r)) + z, -128), 127);
+  }
+  return make_uint2(pack_i8x4(q[0], q[1], q[2], q[3]), pack_i8x4(q[4], q[5], q[6], q[7]));
+}
+
+// ------------------------------------------------------------ per token
+// G threads per row (32 = one warp, or 256 = the whole block), VPT 16-byte
+// chunks (8 bf16) per thread held in registers, so X is read exactly once.
+template <int G, int VPT>
+__global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__restrict__ X,
+                                                              int64_t M, int64_t K, int64_t ldx,
+                                                              int8_t *__restrict__ Xq,
+                                                              float *__restrict__ S_x) {
+  constexpr int R = 256 / G;  // rows per block
+  __shared__ uint32_t red[8];
+  const int tid = threadIdx.x;
+  const int g = tid / G;  // row slot in this block
+  const int t = tid % G;  // thread within the row group
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * R + g;
+  const int64_t chunks = K >> 3;
+  const bool row_ok = m < M;
+  const uint16_t *xrow = X + m * ldx;
+
+  uint4 v[VPT];
+  uint32_t amax = 0;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int64_t c = t + static_cast<int64_t>(j) * G;
+    if (row_ok && c < chunks) {
+      v[j] = __ldcs(reinterpret_cast<const uint4 *>(xrow) + c);
+      amax = absmax_bits_u4(v[j], amax);
+    } else {
+      v[j] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  amax = __reduce_max_sync(0xFFFFFFFFu, amax);
+  if (G > 32) {
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < G / 32; ++w) amax = max(amax, red[w]);
+  }
+  if (!row_ok) return;
+  const float a = __uint_as_float(amax << 16);
+  float r = 0.0f;
+  if (a > 0.0f) r = __fdiv_rn(127.0f, a);
+  if (t == 0) S_x[m] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+  int8_t *qrow = Xq + m * K;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int64_t c = t + static_cast<int64_t>(j) * G;
+    if (c < chunks) reinterpret_cast<uint2 *>(qrow)[c] = quant8_sym(v[j], r);
+  }
+}
+
+template <int G, int VPT>
+static cudaError_t launch_per_token_t(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                      int8_t *Xq, float *S_x, cudaStream_t s) {
+  constexpr int R = 256 / G;
+  const unsigned blocks = static_cast<unsigned>((M + R - 1) / R);
+  quant_per_token_kernel<G, VPT><<<blocks, 256, 0, s>>>(X, M, K, ldx, Xq, S_x);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_per_token(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                   int8_t *Xq, float *S_x, cudaStream_t s) {
+  const int64_t chunks = K / 8;
+  if (chunks <= 32 * 1) return launch_per_token_t<32, 1>(X, M, K, ldx, Xq, S_x, s);
+  if (chunks <= 32 * 2) return launch_per_token_t<32, 2>(X, M, K, ldx, Xq, S_x, s);
+  if (chunks <= 32 * 4) return launch_per_token_t<32, 4>(X, M, K, ldx, Xq, S_x, s);
+  if (chunks <= 32 * 8) return launch_per_token_t<32, 8>(X, M, K, ldx, Xq, S_x, s);
+  if (chunks <= 32 * 16) return launch_per_token_t<32, 16>(X, M, K, ldx, Xq, S_x, s);
+  if (chunks <= 256 * 4) return launch_per_token_t<256, 4>(X, M, K, ldx, Xq, S_x, s);
+  if (chunks <= 256 * 8) return launch_per_token_t<256, 8>(X, M, K, ldx, Xq, S_x, s);
+  if (chunks <= 256 * 16) return launch_per_token_t<256, 16>(X, M, K, ldx, Xq, S_x, s);
+  return launch_per_token_t<256, 32>(X, M, K, ldx, Xq, S_x, s);
+}
+
+// ------------------------------------------------------------ per tensor
+// Grid-stride over 16-byte chunks; r and Z are device scalars.
+__global__ void __launch_bounds__(256) quant_per_tensor_kernel(const uint16_t *__restrict__ X,
+                                                               int64_t M, int64_t K, int64_t ldx,
+                                                               const float *__restrict__ r_ptr,
+                                                               const int32_t *__restrict__ Z_ptr,
+                                                               int8_t *__restrict__ Xq) {
+  const float r = *r_ptr;
+  const int z = *Z_ptr;
+  const int64_t cpr = K >> 3;  // chunks per row
+  const int64_t total = M * cpr;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / cpr, c = i - m * cpr;
+    const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(X + m * ldx) + c);
+    reinterpret_cast<uint2 *>(Xq + m * K)[c] = quant8_asym(v, r, z);
+  }
+}
+
+cudaError_t launch_quant_per_tensor(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                    const float *r, const int32_t *Z, int8_t *Xq, int num_sms,
+                                    cudaStream_t s) {
+  const int64_t total = M * (K / 8);
+  int64_t blocks = (total + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  quant_per_tensor_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(X, M, K, ldx, r, Z, Xq);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ calibration
+// Pass 1: every block reduces the largest positive value and the largest
+// magnitude of a negative value; both are >= +0, so their fp32 bit patterns
+// order like unsigned integers and atomicMax on the bits is exact. The two
+// cells are the S and r outputs themselves (zeroed by the host first).
+template <typename T>
+__device__ __forceinline__ float load_f(const T *p);
+template <>
+__device__ __forceinline__ float load_f<uint16_t>(const uint16_t *p) {
+  return __uint_as_float(static_cast<uint32_t>(__ldg(p)) << 16);
+}
+template <>
+__device__ __forceinline__ float load_f<float>(const float *p) {
+  return __ldg(p);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) calibrate_minmax_kernel(const T *__restrict__ X, int64_t T_,
+                                                               int64_t K, int64_t ldx,
+                                                               uint32_t *hi_cell,
+                                                               uint32_t *neg_lo_cell) {
+  __shared__ uint32_t sh[2][8];
+  uint32_t hi = 0, nlo = 0;
+  const int64_t total = T_ * K;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / K, k = i - t * K;
+    const float v = load_f<T>(X + t * ldx + k);
+    if (v > 0.0f) hi = max(hi, __float_as_uint(v));
+    if (v < 0.0f) nlo = max(nlo, __float_as_uint(-v));
+  }
+  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+  nlo = __reduce_max_sync(0xFFFFFFFFu, nlo);
+  if ((threadIdx.x & 31) == 0) {
+    sh[0][threadIdx.x >> 5] = hi;
+    sh[1][threadIdx.x >> 5] = nlo;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w) {
+      hi = max(hi, sh[0][w]);
+      nlo = max(nlo, sh[1][w]);
+    }
+    hi = max(hi, sh[0][0]);
+    nlo = max(nlo, sh[1][0]);
+    if (hi) atomicMax(hi_cell, hi);
+    if (nlo) atomicMax(neg_lo_cell, nlo);
+  }
+}
+
+// Pass 2 (one thread): S = (hi - lo)/255, r = 255/(hi - lo),
+// Z = clamp(-128 - rne(lo * r), -128, 127); all-zero data gives S = r = 1, Z = 0.
+__global__ void calibrate_finalize_kernel(float *S, float *r, int32_t *Z) {
+  const float hi = __uint_as_float(*reinterpret_cast<uint32_t *>(S));
+  const float nlo = __uint_as_float(*reinterpret_cast<uint32_t *>(r));
+  const float lo = nlo > 0.0f ? -nlo : 0.0f;
+  if (hi == lo) {
+    *S = 1.0f;
+    *r = 1.0f;
+    *Z = 0;
+    return;
+  }
+  const float d = __fsub_rn(hi, lo);
+  const float rr = __fdiv_rn(255.0f, d);
+  *S = __fdiv_rn(d, 255.0f);
+  *r = rr;
+  *Z = min(max(-128 - rne_clamped(__fmul_rn(lo, rr)), -128), 127);
+}
+
+cudaError_t launch_calibrate(const void *X, w8a8_dtype dt, int64_t T, int64_t K, int64_t ldx,
+                             float *S, float *r, int32_t *Z, int num_sms, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(S, 0, sizeof(float), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(r, 0, sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  const int64_t total = T * K;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > static_cast<int64_t>(num_sms) * 4) blocks = static_cast<int64_t>(num_sms) * 4;
+  if (dt == W8A8_BF16)
+    calibrate_minmax_kernel<uint16_t><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<const uint16_t *>(X), T, K, ldx, reinterpret_cast<uint32_t *>(S),
+        reinterpret_cast<uint32_t *>(r));
+  else
+    calibrate_minmax_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<const float *>(X), T, K, ldx, reinterpret_cast<uint32_t *>(S),
+        reinterpret_cast<uint32_t *>(r));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  calibrate_finalize_kernel<<<1, 1, 0, s>>>(S, r, Z);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ weights
+// One block per 32 output channels (columns of W [K, N]). Pass 1: column
+// absmax. Pass 2: quantize 64-row slabs, transpose through shared memory so
+// that Wq [N, K] is written along K, and accumulate colsum.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_weight_kernel(const T *__restrict__ W, int64_t K,
+                                                           int64_t N, int64_t ldw,
+                                                           int8_t *__restrict__ Wq,
+                                                           float *__restrict__ s_w,
+                                                           int32_t *__restrict__ colsum) {
+  __shared__ float red[8][32];
+  __shared__ int32_t csum[8][32];
+  __shared__ __align__(16) int8_t tile[32][64 + 16];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int64_t n = n0 + tx;
+  const bool col_ok = n < N;
+
+  float a = 0.0f;
+  if (col_ok)
+    for (int64_t k = ty; k < K; k += 8) a = fmaxf(a, fabsf(load_f<T>(W + k * ldw + n)));
+  red[ty][tx] = a;
+  __syncthreads();
+  a = red[0][tx];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w][tx]);
+  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+  if (ty == 0 && col_ok) s_w[n] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+
+  int32_t cs = 0;
+  const int wr = threadIdx.x >> 3;  // output row (channel) this thread writes, 0..31
+  const int wp = threadIdx.x & 7;   // 8-byte piece of the 64-byte slab row
+  for (int64_t k0 = 0; k0 < K; k0 += 64) {
+    for (int kk = ty; kk < 64; kk += 8) {
+      const int64_t k = k0 + kk;
+      int q = 0;
+      if (col_ok && k < K) q = min(max(rne_clamped(__fmul_rn(load_f<T>(W + k * ldw + n), r)), -127), 127);
+      cs += q;
+      tile[tx][kk] = static_cast<int8_t>(q);
+    }
+    __syncthreads();
+    const int64_t nw = n0 + wr, kw = k0 + wp * 8;
+    if (nw < N && kw < K)
+      *reinterpret_cast<uint2 *>(Wq + nw * K + kw) = *reinterpret_cast<const uint2 *>(&tile[wr][wp * 8]);
+    __syncthreads();
+  }
+  csum[ty][tx] = cs;
+  __syncthreads();
+  if (ty == 0 && col_ok) {
+    int32_t s = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += csum[w][tx];
+    colsum[n] = s;
+  }
+}
+
+cudaError_t launch_quant_weight(const void *W, w8a8_dtype dt, int64_t K, int64_t N, int64_t ldw,
+                                int8_t *Wq, float *s_w, int32_t *colsum, cudaStream_t s) {
+  const unsigned blocks = static_cast<unsigned>((N + 31) / 32);
+  if (dt == W8A8_BF16)
+    quant_weight_kernel<uint16_t><<<blocks, 256, 0, s>>>(static_cast<const uint16_t *>(W), K, N,
+                                                         ldw, Wq, s_w, colsum);
+  else
+    quant_weight_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float *>(W), K, N, ldw,
+                                                      Wq, s_w, colsum);
+  return cudaGetLastError();
+}
+
+}  // namespace w8a8

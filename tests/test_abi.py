@@ -1,0 +1,102 @@
+"""The C ABI on a host without a GPU: the library loads, exports every symbol
+include/w8a8.h declares, and rejects bad arguments on the host before any
+CUDA call (fake pointers are never dereferenced)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from int8_gemm_token_b200 import w8a8
+
+GOOD = 0x10000  # a 16-byte aligned fake device address (never dereferenced)
+ODD = 0x10008
+
+
+@pytest.fixture(scope="module")
+def L():
+    return w8a8.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = w8a8.header_symbols()
+    assert len(names) >= 13
+    out = subprocess.run(["nm", "-D", "--defined-only", w8a8.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(L, n)
+    assert set(w8a8._SIGNATURES) == set(names)
+
+
+def test_status_strings(L):
+    for code, name in [(0, "W8A8_OK"), (1, "W8A8_ERR_INVALID_ARG"), (2, "W8A8_ERR_MISALIGNED"),
+                       (3, "W8A8_ERR_UNSUPPORTED_SHAPE"), (4, "W8A8_ERR_UNSUPPORTED_DTYPE"),
+                       (6, "W8A8_ERR_DEVICE_TIMEOUT"), (7, "W8A8_ERR_OUTLIER_OVERFLOW"),
+                       (9, "W8A8_ERR_WORKSPACE"), (10, "W8A8_ERR_NO_DEVICE"), (1234, "W8A8_ERR_UNKNOWN")]:
+        assert w8a8.status_string(code) == name
+
+
+def test_quant_per_token_host_checks(L):
+    f = L.w8a8_quant_per_token
+    assert f(GOOD, 4, 15, 16, GOOD, GOOD, None) == 3          # K not a multiple of 16
+    assert f(GOOD, 4, 65536 + 16, 65552, GOOD, GOOD, None) == 3
+    assert f(GOOD, 4, 0, 16, GOOD, GOOD, None) == 1
+    assert f(GOOD, -1, 16, 16, GOOD, GOOD, None) == 1
+    assert f(GOOD, 4, 32, 16, GOOD, GOOD, None) == 1          # ldx < K
+    assert f(None, 4, 32, 32, GOOD, GOOD, None) == 1
+    assert f(ODD, 4, 32, 32, GOOD, GOOD, None) == 2
+    assert f(GOOD, 4, 32, 36, GOOD, GOOD, None) == 2          # rows not 16-byte aligned
+    assert f(GOOD, 4, 32, 32, None, GOOD, None) == 1
+    assert f(GOOD, 0, 32, 32, None, None, None) == 0          # empty: nothing to do
+
+
+def test_gemm_host_checks(L):
+    f = L.w8a8_gemm_dequant
+    args = dict(Xq=GOOD, S_x=GOOD, per_row=1, Z=None, Wq=GOOD, s_w=GOOD, colsum=None, bias=None,
+                M=8, N=8, K=64, out=GOOD, dt=0, ws=None, wsb=0, stream=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(*a.values())
+    assert call(K=40) == 3
+    assert call(dt=7) == 4
+    assert call(Wq=None) == 1
+    assert call(Z=GOOD, colsum=None) == 1
+    assert call(out=ODD) == 2
+    assert call(bias=ODD) == 2
+    assert call(M=0) == 0 and call(N=0) == 0
+    assert call(M=-2) == 1
+
+
+def test_linear_static_workspace_check(L):
+    f = L.w8a8_linear_static
+    # X, M, K, ldx, S, r, Z, Wq, s_w, colsum, bias, N, out, dt, ws, wsb, stream
+    assert f(GOOD, 4, 64, 64, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, None, 8, GOOD, 0, None, 0, None) == 9
+    assert f(GOOD, 4, 64, 64, GOOD, GOOD, None, GOOD, GOOD, GOOD, None, 8, GOOD, 0, GOOD, 4096, None) == 1
+
+
+def test_other_entry_points_host_checks(L):
+    assert L.w8a8_quant_weight_per_channel(GOOD, 5, 64, 8, 8, GOOD, GOOD, GOOD, None) == 4
+    assert L.w8a8_quant_weight_per_channel(GOOD, 1, 64, 8, 4, GOOD, GOOD, GOOD, None) == 1
+    assert L.w8a8_quant_weight_per_channel(GOOD + 1, 0, 64, 3, 3, GOOD, GOOD, GOOD, None) == 2  # odd bf16 address
+    assert L.w8a8_quant_weight_per_channel(GOOD, 0, 64, 3, 3, GOOD + 4, GOOD, GOOD, None) == 2  # Wq rows
+    assert L.w8a8_calibrate_static(GOOD, 0, 0, 16, 16, GOOD, GOOD, GOOD, None) == 1
+    assert L.w8a8_calibrate_static(GOOD, 3, 4, 16, 16, GOOD, GOOD, GOOD, None) == 4
+    assert L.w8a8_quant_per_tensor(GOOD, 4, 64, 64, None, GOOD, GOOD, None) == 1
+    assert L.int8_mixed_decomp_gemm(GOOD, GOOD, GOOD, GOOD, GOOD, 8, GOOD, GOOD, GOOD, 8, None,
+                                    8, 8, 64, GOOD, 2, None) == 4  # int32 output not offered here
+    assert L.int8_mixed_decomp_gemm(GOOD, GOOD, GOOD, GOOD, GOOD, 5000, GOOD, GOOD, GOOD, 8, None,
+                                    8, 8, 64, GOOD, 0, None) == 1
+    assert L.w8a8_debug_wait_timeout_selftest(10, None) == 1
+    st = ctypes.c_int32(0)
+    assert L.w8a8_check_device_error(None, None) == 1
+
+
+def test_valid_call_without_a_gpu_reports_no_device(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert L.w8a8_quant_per_token(GOOD, 4, 32, 32, GOOD, GOOD, None) == 10
+    assert w8a8.w8a8_gemm_workspace_size(4, 8, 64) >= 4 * 64
+    assert w8a8.lib().int8_outlier_split_workspace_size(8192) >= 8192 // 8

@@ -1,0 +1,194 @@
+"""CUDA path vs the CPU oracle, element by element, on seeded inputs.
+
+Integers (codes, zero points, column sums, int32 accumulators) and scales
+must match bit for bit. Outputs must match too: the epilogue performs the
+same fp32 operations in the same order as the oracle (int->float RN,
+S_x*s_w RN, one fmaf, bf16 RNE), so bf16 and fp32 outputs are compared for
+exact equality -- stricter than the 1e-3 relative bound the layer is held to.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from int8_gemm_token_b200 import synth
+from int8_gemm_token_b200 import w8a8 as W
+from tests.gpu_util import dev, dev_bf16, diff_report, host, host_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    yield
+    assert W.w8a8_check_device_error() == 0
+
+
+def assert_same(gpu, ref, what):
+    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    if gpu.dtype == np.float32:
+        eq = (gpu.view(np.uint32) == ref.view(np.uint32))
+    else:
+        eq = gpu == ref
+    assert eq.all(), f"{what}: " + diff_report(gpu, ref)
+
+
+# ------------------------------------------------------------ quantizers
+@pytest.mark.parametrize("M,K,ld_pad", [(16, 256, 0), (1, 16, 0), (3, 48, 8), (130, 4096, 0),
+                                        (7, 4112, 0), (33, 11008, 16), (5, 65536, 0), (2, 8192 + 16, 0)])
+def test_quant_per_token_bit_exact(M, K, ld_pad):
+    rng = np.random.default_rng(M * 7 + K)
+    X = synth.activations(rng, M, K, with_outliers=K >= 64)
+    if M > 2:
+        X[1] = 0  # an all-zero token
+    Xd_full = dev_bf16(np.pad(X, ((0, 0), (0, ld_pad))))
+    Xd = Xd_full[:, :K]
+    Xq, S = W.w8a8_quant_per_token(Xd)
+    rq, rS = oracle.quant_per_token(X)
+    assert_same(host(Xq), rq, "Xq")
+    assert_same(host(S), rS, "S_x")
+
+
+def test_quant_per_token_ties():
+    X = synth.bf16_bits(np.array([[254, 1, -1, 3, 5, -5, 7, 9] + [0] * 8], np.float32))
+    Xq, S = W.w8a8_quant_per_token(dev_bf16(X))
+    assert list(host(Xq)[0, :8]) == [127, 0, 0, 2, 2, -2, 4, 4]
+
+
+@pytest.mark.parametrize("M,K", [(1, 4096), (32, 4096), (4096, 4096), (5, 48)])
+def test_calibrate_and_quant_per_tensor_bit_exact(M, K):
+    case = synth.decode_static(M=min(M, 64), N=16, K=K, seed=M)
+    S, r, Z = W.w8a8_calibrate_static(dev_bf16(case.Xcal))
+    rS, rr, rZ = oracle.calibrate_static(case.Xcal)
+    assert host(S)[0] == rS and host(r)[0] == rr and host(Z)[0] == rZ
+    X = case.X if M <= 64 else synth.calibration_tokens(np.random.default_rng(5), M, K)
+    Xq = W.w8a8_quant_per_tensor(dev_bf16(X), r, Z)
+    assert_same(host(Xq), oracle.quant_per_tensor(X, rr, rZ), "Xq")
+
+
+def test_calibrate_signed_fp32_and_zero():
+    rng = np.random.default_rng(9)
+    Xcal = synth.bits_to_f32(synth.activations(rng, 100, 200, with_outliers=True))
+    S, r, Z = W.w8a8_calibrate_static(dev(Xcal))
+    assert (host(S)[0], host(r)[0], host(Z)[0]) == oracle.calibrate_static(Xcal)
+    S, r, Z = W.w8a8_calibrate_static(dev(np.zeros((3, 50), np.float32)))
+    assert (host(S)[0], host(r)[0], host(Z)[0]) == (1.0, 1.0, 0)
+
+
+@pytest.mark.parametrize("K,N,dtype", [(256, 512, "f32"), (4096, 520, "f32"), (400, 33, "bf16"),
+                                       (16, 8, "bf16"), (11008, 96, "f32")])
+def test_weight_quant_bit_exact(K, N, dtype):
+    rng = np.random.default_rng(K + N)
+    Wf = synth.weight(rng, K, N)
+    Wf[:, 1] = 0.0
+    if dtype == "bf16":
+        Wh = synth.bf16_bits(Wf)
+        Wd = dev_bf16(Wh)
+    else:
+        Wh = Wf
+        Wd = dev(Wf)
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(Wd)
+    rq, rs, rc = oracle.quant_weight_per_channel(Wh)
+    assert_same(host(Wq), rq, "Wq")
+    assert_same(host(s_w), rs, "s_w")
+    assert_same(host(cs), rc, "colsum")
+
+
+# ------------------------------------------------------------ GEMM
+def _rand_case(M, N, K, seed):
+    rng = np.random.default_rng(seed)
+    X = synth.activations(rng, M, K, with_outliers=True)
+    Wf = synth.weight(rng, K, N)
+    b = synth.bias(rng, N)
+    return X, Wf, b
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 512, 256), (128, 256, 128), (300, 520, 400), (1, 40, 16),
+                                   (257, 1000, 4096), (129, 257, 144)])
+def test_gemm_int32_accumulator_bit_exact(M, N, K):
+    X, Wf, b = _rand_case(M, N, K, M + N + K)
+    rq, rS = oracle.quant_per_token(X)
+    wq, ws, wc = oracle.quant_weight_per_channel(Wf)
+    acc = W.w8a8_gemm_dequant(dev(rq), dev(rS), dev(wq), dev(ws), out_dtype=torch.int32)
+    assert_same(host(acc), oracle.gemm_i64(rq, wq).astype(np.int32), "acc")
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 400), (200, 264, 512)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_prefill_linear_bit_exact(M, N, K, out_dtype):
+    X, Wf, b = _rand_case(M, N, K, 3 * M + N)
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(Wf))
+    Xq, S_x = W.w8a8_quant_per_token(dev_bf16(X))
+    out = W.w8a8_gemm_dequant(Xq, S_x, Wq, s_w, bias=dev(b), out_dtype=out_dtype)
+    rwq, rws, _ = oracle.quant_weight_per_channel(Wf)
+    _, _, _, y = oracle.linear_prefill(X, rwq, rws, bias=b)
+    if out_dtype == torch.bfloat16:
+        assert_same(host_bf16(out), oracle.f32_to_bf16(y), "out")
+    else:
+        assert_same(host(out), y, "out")
+
+
+def test_zero_point_path_and_raw_corrected_accumulator():
+    M, N, K = 40, 300, 256
+    case = synth.decode_static(M=M, N=N, K=K, seed=3)
+    rS, rr, rZ = oracle.calibrate_static(case.Xcal)
+    rxq = oracle.quant_per_tensor(case.X, rr, rZ)
+    rwq, rws, rwc = oracle.quant_weight_per_channel(case.W)
+    S, r, Z = W.w8a8_calibrate_static(dev_bf16(case.Xcal))
+    Xq = W.w8a8_quant_per_tensor(dev_bf16(case.X), r, Z)
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(case.W))
+    c = W.w8a8_gemm_dequant(Xq, S, Wq, s_w, colsum=cs, Z=Z, out_dtype=torch.int32)
+    acc = oracle.gemm_i64(rxq, rwq)
+    assert_same(host(c), (acc - int(rZ) * rwc.astype(np.int64)[None, :]).astype(np.int32), "acc - Z colsum")
+    y = W.w8a8_gemm_dequant(Xq, S, Wq, s_w, colsum=cs, Z=Z, out_dtype=torch.float32)
+    assert_same(host(y), oracle.epilogue(acc, rS, rws, colsum=rwc, Z=rZ), "y")
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 32])
+@pytest.mark.parametrize("N", [4096, 11008])
+def test_decode_linear_static_bit_exact(M, N):
+    case = synth.decode_static(M=M, N=N, seed=0)
+    S, r, Z = W.w8a8_calibrate_static(dev_bf16(case.Xcal))
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(case.W))
+    out = W.w8a8_linear_static(dev_bf16(case.X), S, r, Z, Wq, s_w, cs)
+    rS, rr, rZ = oracle.calibrate_static(case.Xcal)
+    rwq, rws, rwc = oracle.quant_weight_per_channel(case.W)
+    rxq, _, y = oracle.linear_decode(case.X, rr, rZ, rS, rwq, rws, rwc)
+    assert (rxq == 127).any() and (rxq == -128).any()  # the 1% pushed past the range saturates
+    assert_same(host_bf16(out), oracle.f32_to_bf16(y), "out")
+
+
+def test_prefill_7b_full_size_sampled():
+    """The full 2048 x 4096 x 11008 workload in the launch configuration the
+    benchmark uses; Xq, S_x, Wq, s_w, colsum are compared in full, outputs on
+    a sample of 96 rows x 96 columns that the oracle computes one by one."""
+    case = synth.prefill_7b(0)
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(case.W))
+    Xq, S_x = W.w8a8_quant_per_token(dev_bf16(case.X))
+    out = W.w8a8_gemm_dequant(Xq, S_x, Wq, s_w, bias=dev(case.bias))
+    rxq, rS = oracle.quant_per_token(case.X)
+    rwq, rws, rwc = oracle.quant_weight_per_channel(case.W)
+    assert_same(host(Xq), rxq, "Xq")
+    assert_same(host(S_x), rS, "S_x")
+    assert_same(host(Wq), rwq, "Wq")
+    assert_same(host(s_w), rws, "s_w")
+    assert_same(host(cs), rwc, "colsum")
+    rng = np.random.default_rng(99)
+    rows = np.sort(rng.choice(2048, 96, replace=False))
+    rows[-1] = 2047
+    cols = np.sort(rng.choice(11008, 96, replace=False))
+    cols[-1] = 11007
+    acc = oracle.gemm_i64(rxq[rows], rwq[cols])
+    y = oracle.epilogue(acc, rS[rows], rws[cols], bias=case.bias[cols])
+    got = host_bf16(out)[np.ix_(rows, cols)]
+    assert_same(got, oracle.f32_to_bf16(y), "sampled out")
+
+
+# ------------------------------------------------------------ failure path
+def test_bounded_wait_reports_timeout_and_device_stays_usable():
+    W.w8a8_debug_wait_timeout_selftest(2_000_000)
+    assert W.w8a8_check_device_error() == 6  # W8A8_ERR_DEVICE_TIMEOUT
+    assert W.w8a8_check_device_error() == 0  # cleared
+    X = synth.activations(np.random.default_rng(0), 4, 64)
+    Xq, S = W.w8a8_quant_per_token(dev_bf16(X))
+    assert_same(host(Xq), oracle.quant_per_token(X)[0], "Xq after timeout")
