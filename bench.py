@@ -318,8 +318,7 @@ def bench_decode(args, dev, rank, peaks, max_over_ranks, barrier):
     Wq, s_w, cs = W.w8a8_quant_weight_per_channel(torch.from_numpy(case.W).to(dev))
     for i in range(n_w):
         ws.append((Wq.clone(), s_w.clone(), cs.clone(), torch.empty((DEC_M, DEC_N), dtype=torch.bfloat16, device=dev)))
-    wsz = W.w8a8_gemm_workspace_size(DEC_M, DEC_N, DEC_K)
-    work = torch.empty((max(wsz, 1),), dtype=torch.uint8, device=dev)
+    work = W.new_workspace(DEC_M, DEC_N, DEC_K, device=dev)
     stream = torch.cuda.current_stream()
     steps = max(args.steps, 20)
     for i in range(max(args.warmup, 3)):

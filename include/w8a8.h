@@ -148,7 +148,14 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
  *   s_w     device fp32 [N];  bias device fp32 [N] or NULL
  *   out     device [M, N] dense, out_dtype W8A8_BF16, W8A8_FP32 or W8A8_I32
  *   workspace/workspace_bytes: device scratch of at least
- *           w8a8_gemm_workspace_size(M, N, K) bytes (NULL allowed when it is 0)
+ *           w8a8_gemm_workspace_size(M, N, K) bytes (NULL allowed when it is 0).
+ * M <= 32 (Decode-shaped) runs a split-K kernel that keeps per-tile counters
+ * and int32 partial sums at the start of the workspace (the first
+ * ceil(ceil(N/128) * 4 / 256) * 256 + ceil(N/128) * 16384 bytes). That region
+ * must be zero before the first call that uses the workspace, and every call
+ * that completes leaves it zero again, so one zero-filled workspace serves
+ * every later call. Calls that overlap on the GPU must not share a workspace;
+ * after a call that recorded a device error, zero the workspace again.
  */
 w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_per_row,
                               const int32_t *Z, const int8_t *Wq, const float *s_w,
@@ -157,14 +164,20 @@ w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
                               size_t workspace_bytes, void *stream);
 
 /* Bytes of device workspace w8a8_gemm_dequant / w8a8_linear_static need for
- * this shape (0 when none). */
+ * this shape (enough for either call): for M <= 32 the tile counters
+ * (ceil(N/128) * 4 bytes rounded up to 256), the split-K partial sums
+ * (ceil(N/128) * 16 KiB), then M*K bytes (rounded up to 256) for the
+ * statically quantized activation of w8a8_linear_static; for M > 32 only the
+ * last part. */
 size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
- * Fused Decode linear: static per-tensor quantization of bf16 X done inside
- * the GEMM kernel (no separate launch), then the GEMM and the zero-point
- * corrected epilogue. Same result as w8a8_quant_per_tensor followed by
- * w8a8_gemm_dequant with s_x_per_row = 0.
+ * Decode linear in one call: static per-tensor quantization of bf16 X into
+ * the workspace, then the GEMM with the zero-point corrected epilogue. Same
+ * result as w8a8_quant_per_tensor followed by w8a8_gemm_dequant with
+ * s_x_per_row = 0. For M <= 32 the GEMM kernel is launched with programmatic
+ * dependent launch, so it streams the weight while the quantization kernel
+ * runs and reads the quantized activation once that kernel has finished.
  * Source: PDMIX glossary §2.2 (Decode has few tokens and is latency bound, so
  * a per-step quantization launch would be visible overhead) and §2.3 eq.
  * Q_decode; the hardware-acceleration chapter's note that decode is memory
@@ -195,10 +208,12 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
  *   n_out        device int32 scalar, written: the number n of outlier columns
  *   Xo           device bf16 [M, cap] dense, written: Xo[m, j] = X[m, idx[j]]
  *                for j < min(n, cap)
- *   workspace    device, >= int8_outlier_split_workspace_size(K) bytes
+ *   workspace    device, >= int8_outlier_split_workspace_size(K) bytes, 4-byte
+ *                aligned (a K-bit column bitmap; the call clears it itself)
  * cap is in [0, 4096]. n > cap sets W8A8_ERR_OUTLIER_OVERFLOW in the device
  * status word; the outputs then describe only the first cap outliers (the
  * others are still zeroed in Xq, so the result would be wrong: check it).
+ * M == 0 writes nothing.
  */
 w8a8_status int8_outlier_split(const void *X, int64_t M, int64_t K, int64_t ldx, float threshold,
                                int32_t cap, int8_t *Xq, float *S_x, int32_t *outlier_idx,

@@ -84,8 +84,8 @@ w8a8_status check_bf16_rows(const void *X, int64_t M, int64_t K, int64_t ldx) {
 
 }  // namespace
 
-bool encode_tmap_2d_u8(void *map, const void *base, uint64_t inner, uint64_t outer,
-                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+bool encode_tmap_2d(void *map, const void *base, TmapType type, uint64_t inner, uint64_t outer,
+                    uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
   std::call_once(g_encode_once, [] {
     void *fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -100,9 +100,10 @@ bool encode_tmap_2d_u8(void *map, const void *base, uint64_t inner, uint64_t out
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
-                        const_cast<void *>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = g_encode(static_cast<CUtensorMap *>(map),
+                        type == TmapType::kU8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -185,11 +186,17 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
                                            d->sm_count, static_cast<cudaStream_t>(stream)));
 }
 
+// Decode-shaped calls (at most this many tokens) take the stream-K kernel.
+constexpr int64_t kDecodeMaxM = 32;
+
+static size_t align256(int64_t n) { return static_cast<size_t>(((n + 255) / 256) * 256); }
+
 size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
-  (void)N;
-  if (M <= 0 || K <= 0) return 0;
-  // w8a8_linear_static keeps the statically quantized activation here.
-  return static_cast<size_t>(((M * K + 255) / 256) * 256);
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  // w8a8_linear_static keeps the statically quantized activation here (M*K bytes);
+  // the decode-shaped kernel (M <= 32) puts its tile counters and partial sums first.
+  if (M <= kDecodeMaxM) return decode_counters_bytes(N) + decode_partials_bytes(N) + align256(M * K);
+  return align256(M * K);
 }
 
 static w8a8_status check_gemm_common(const int8_t *Xq, const int8_t *Wq, const float *s_w,
@@ -212,11 +219,14 @@ w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
                               const int32_t *colsum, const float *bias, int64_t M, int64_t N,
                               int64_t K, void *out, w8a8_dtype out_dtype, void *workspace,
                               size_t workspace_bytes, void *stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (w8a8_status s = check_gemm_common(Xq, Wq, s_w, bias, colsum, M, N, K, out, out_dtype)) return s;
   if (M == 0 || N == 0) return W8A8_OK;
   if (!S_x || (Z && !colsum)) return W8A8_ERR_INVALID_ARG;
+  const bool decode = M <= kDecodeMaxM;
+  if (decode) {
+    if (!workspace || workspace_bytes < w8a8_gemm_workspace_size(M, N, K)) return W8A8_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return W8A8_ERR_MISALIGNED;
+  }
   DeviceInfo *d;
   if (w8a8_status s = device_info(&d)) return s;
   EpilogueArgs ep;
@@ -228,6 +238,9 @@ w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
   ep.bias = bias;
   ep.out = out;
   ep.out_dtype = out_dtype;
+  if (decode)  // ordinary stream order: the previous kernel may have written the weights
+    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, workspace, false, d->sm_count, d->status,
+                                        static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_gemm_tc(Xq, Wq, M, N, K, ep, false, d->sm_count, d->status,
                                   static_cast<cudaStream_t>(stream)));
 }
@@ -252,10 +265,6 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
   DeviceInfo *d;
   if (w8a8_status s = device_info(&d)) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int8_t *Xq = static_cast<int8_t *>(workspace);
-  cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq,
-                                          d->sm_count, st);
-  if (e != cudaSuccess) return W8A8_ERR_CUDA;
   EpilogueArgs ep;
   ep.S_x = S;
   ep.s_x_per_row = 0;
@@ -265,21 +274,43 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
   ep.bias = bias;
   ep.out = out;
   ep.out_dtype = out_dtype;
+  if (M <= kDecodeMaxM) {
+    // Static quantization into the workspace, then the decode GEMM launched with
+    // programmatic dependent launch: its weight stream starts while the
+    // quantization runs, and it reads the quantized activation after it.
+    int8_t *Xq = static_cast<int8_t *>(workspace) + decode_counters_bytes(N) + decode_partials_bytes(N);
+    cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq, d->sm_count, st);
+    if (e != cudaSuccess) return W8A8_ERR_CUDA;
+    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, workspace, true, d->sm_count, d->status, st));
+  }
+  int8_t *Xq = static_cast<int8_t *>(workspace);
+  cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq,
+                                          d->sm_count, st);
+  if (e != cudaSuccess) return W8A8_ERR_CUDA;
   return from_cuda(launch_gemm_tc(Xq, Wq, M, N, K, ep, false, d->sm_count, d->status, st));
 }
 
 size_t int8_outlier_split_workspace_size(int64_t K) {
   if (K <= 0) return 0;
-  return static_cast<size_t>(((K + 31) / 32) * 4 + 256);
+  return align256(static_cast<int64_t>(outlier_workspace_bytes(K)));
 }
 
 w8a8_status int8_outlier_split(const void *X, int64_t M, int64_t K, int64_t ldx, float threshold,
                                int32_t cap, int8_t *Xq, float *S_x, int32_t *outlier_idx,
                                int32_t *n_out, void *Xo, void *workspace, size_t workspace_bytes,
                                void *stream) {
-  (void)X; (void)M; (void)K; (void)ldx; (void)threshold; (void)cap; (void)Xq; (void)S_x;
-  (void)outlier_idx; (void)n_out; (void)Xo; (void)workspace; (void)workspace_bytes; (void)stream;
-  return W8A8_ERR_NOT_IMPLEMENTED;
+  if (w8a8_status s = check_bf16_rows(X, M, K, ldx)) return s;
+  if (cap < 0 || cap > 4096) return W8A8_ERR_INVALID_ARG;
+  if (M == 0) return W8A8_OK;
+  if (!Xq || !S_x || !n_out || (cap > 0 && (!outlier_idx || !Xo))) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(Xq) || (Xo && (reinterpret_cast<uintptr_t>(Xo) & 1u))) return W8A8_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < int8_outlier_split_workspace_size(K)) return W8A8_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 3u) != 0) return W8A8_ERR_MISALIGNED;
+  DeviceInfo *d;
+  if (w8a8_status s = device_info(&d)) return s;
+  return from_cuda(launch_outlier_split(static_cast<const uint16_t *>(X), M, K, ldx, threshold, cap, Xq, S_x,
+                                        outlier_idx, n_out, static_cast<uint16_t *>(Xo), workspace, d->status,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 w8a8_status int8_mixed_decomp_gemm(const int8_t *Xq, const float *S_x, const void *Xo,

@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
+  __syncwarp();  // bar.sync is warp-aligned: reconverge after the single-thread set-up
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
@@ -347,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
+  __syncwarp();  // lanes of the producer and MMA warps reconverge before the CTA barrier
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -359,11 +361,11 @@ cudaError_t launch_tc_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N
                         const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
   using Cfg = TcConfig<BN, STAGES>;
   alignas(64) CUtensorMap tmA, tmB;
-  if (!encode_tmap_2d_u8(&tmA, Xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                         static_cast<uint64_t>(K), kBK, kBM))
+  if (!encode_tmap_2d(&tmA, Xq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                      static_cast<uint64_t>(K), kBK, kBM, true))
     return cudaErrorInvalidValue;
-  if (!encode_tmap_2d_u8(&tmB, Wq, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
-                         static_cast<uint64_t>(K), kBK, BN))
+  if (!encode_tmap_2d(&tmB, Wq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                      static_cast<uint64_t>(K), kBK, BN, true))
     return cudaErrorInvalidValue;
   auto kern = gemm_i8_tc_kernel<BN, STAGES, MIXED>;
   // per function and per device; cheap enough to repeat on every launch

@@ -48,8 +48,33 @@ cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_t s);
 
-// Driver entry point for tensor-map encoding (resolved once per process).
-bool encode_tmap_2d_u8(void *map, const void *base, uint64_t inner, uint64_t outer,
-                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+// Decode-shaped GEMM (M <= 32): stream-K over the weight. The workspace holds
+// the per-tile counters (decode_counters_bytes(N)) and then the per-tile int32
+// partial sums (decode_partials_bytes(N)); both must be zero before the first
+// call and every completed call leaves them zero. pdl = true lets the kernel
+// start while the previous kernel in the stream runs: it streams weights at
+// once and waits for that kernel before reading Xq, the workspace or `out`
+// (so the previous kernel must not write Wq, s_w, colsum or bias).
+cudaError_t launch_gemm_decode(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
+                               const EpilogueArgs &ep, void *workspace, bool pdl, int num_sms, int32_t *status,
+                               cudaStream_t s);
+size_t decode_counters_bytes(int64_t N);
+size_t decode_partials_bytes(int64_t N);
+int decode_grid(int64_t N, int64_t K, int num_sms);
+
+// LLM.int8() outlier split: column-flag pass into a K-bit bitmap in
+// `workspace` (outlier_workspace_bytes(K); zeroed by the launcher), then the
+// masked per-row quantization and outlier gather.
+cudaError_t launch_outlier_split(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, float threshold, int32_t cap,
+                                 int8_t *Xq, float *S_x, int32_t *idx, int32_t *n_out, uint16_t *Xo, void *workspace,
+                                 int32_t *status, cudaStream_t s);
+size_t outlier_workspace_bytes(int64_t K);
+
+// 2-D tensor map (driver entry point resolved once per process): inner and
+// outer extents in elements, row stride in bytes, box in elements; swizzle128
+// selects the 128-byte swizzle (box inner extent must then be 128 bytes).
+enum class TmapType { kU8, kBF16 };
+bool encode_tmap_2d(void *map, const void *base, TmapType type, uint64_t inner, uint64_t outer,
+                    uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
 
 }  // namespace w8a8

@@ -1,0 +1,249 @@
+// outlier.cu -- LLM.int8() outlier split (HBM-bound, two passes over X).
+//
+// What it computes: LLM.int8() paper summary, architecture figure, 16-bit
+// decomposition step (1) (the feature columns of X whose magnitude exceeds the
+// threshold are split off, with the matching rows of W) and the 8-bit
+// vector-wise steps (1)-(2) for the remaining columns (row constant C_x,
+// X * 127 / C_x, integers in [-127, 127]); mixed-precision decomposition steps
+// 1-2 (threshold 6.0). Readings: a column is an outlier when any of its
+// entries has |x| > threshold (strict); its entries become 0 in Xq and do not
+// enter the row scale; outlier indices are reported in ascending order.
+//
+// Pass 1 (column flags): each thread owns 8 adjacent columns (one 16-byte
+//   load per row) over a band of rows, keeps the largest magnitude per column
+//   and sets the columns' bits in a K-bit workspace bitmap when it exceeds the
+//   threshold (atomicOr only for outlier columns, so almost never).
+// Pass 2 (rows): every CTA turns the bitmap into the ascending index list
+//   (block-wide popcount scan, in shared memory); CTA 0 publishes it and the
+//   count. Each row is then loaded once into registers (16-byte loads),
+//   outlier columns are masked to zero, the absmax is reduced with warp
+//   shuffles, the row is quantized from registers, and the row's outlier
+//   values are gathered into Xo.
+#include "device.cuh"
+#include "kernels.h"
+
+namespace w8a8 {
+
+namespace {
+
+constexpr int kRowsPerThread = 32;  // pass 1: rows per thread band
+
+// ------------------------------------------------------------------ pass 1
+__global__ void __launch_bounds__(256) outlier_colflag_kernel(const uint16_t *__restrict__ X, int64_t M, int64_t K,
+                                                              int64_t ldx, float threshold,
+                                                              uint32_t *__restrict__ bitmap) {
+  const int64_t groups = K >> 3;  // 8-column groups
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= groups) return;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kRowsPerThread;
+  const int64_t r1 = r0 + kRowsPerThread < M ? r0 + kRowsPerThread : M;
+  uint32_t mx[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // magnitude bits per column
+  const uint4 *p = reinterpret_cast<const uint4 *>(X + r0 * ldx) + g;
+  const int64_t step = ldx >> 3;
+  int64_t r = r0;
+  for (; r + 8 <= r1; r += 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __ldcs(p + i * step);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        mx[2 * j] = max(mx[2 * j], w[j] & 0x7FFFu);
+        mx[2 * j + 1] = max(mx[2 * j + 1], (w[j] >> 16) & 0x7FFFu);
+      }
+    }
+    p += 8 * step;
+  }
+  for (; r < r1; ++r) {
+    const uint4 v = __ldcs(p);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      mx[2 * j] = max(mx[2 * j], w[j] & 0x7FFFu);
+      mx[2 * j + 1] = max(mx[2 * j + 1], (w[j] >> 16) & 0x7FFFu);
+    }
+    p += step;
+  }
+  uint32_t bits = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (__uint_as_float(mx[j] << 16) > threshold) bits |= 1u << j;
+  if (bits) atomicOr(bitmap + ((g * 8) >> 5), bits << ((g * 8) & 31));
+}
+
+// ------------------------------------------------------------------ pass 2
+// Ascending outlier index list from the bitmap, into shared memory (first
+// `cap` entries); returns the total count. All threads of the block call it.
+__device__ int32_t build_outlier_list(const uint32_t *__restrict__ bitmap, int64_t words, int32_t cap,
+                                      int32_t *s_idx, int32_t *s_scan) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int64_t per = (words + nt - 1) / nt;
+  const int64_t w0 = tid * per, w1 = w0 + per < words ? w0 + per : words;
+  int32_t cnt = 0;
+  for (int64_t w = w0; w < w1; ++w) cnt += __popc(__ldcg(bitmap + w));
+  // block exclusive scan of cnt
+  const int lane = tid & 31, warp = tid >> 5;
+  int32_t incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) s_scan[warp] = incl;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t run = 0;
+    for (int i = 0; i < nt / 32; ++i) {
+      const int32_t c = s_scan[i];
+      s_scan[i] = run;
+      run += c;
+    }
+    s_scan[nt / 32] = run;
+  }
+  __syncthreads();
+  int32_t pos = s_scan[warp] + incl - cnt;
+  for (int64_t w = w0; w < w1 && pos < cap; ++w) {
+    uint32_t bitsw = __ldcg(bitmap + w);
+    while (bitsw && pos < cap) {
+      const int b = __ffs(bitsw) - 1;
+      bitsw &= bitsw - 1;
+      s_idx[pos++] = static_cast<int32_t>(w * 32 + b);
+    }
+  }
+  const int32_t total = s_scan[nt / 32];
+  __syncthreads();
+  return total;
+}
+
+// G threads per row (32: one warp per row, 8 rows per block; 256: one row per
+// block), VPT 16-byte chunks per thread held in registers.
+template <int G, int VPT>
+__global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__restrict__ X, int64_t M, int64_t K,
+                                                          int64_t ldx, const uint32_t *__restrict__ bitmap,
+                                                          int32_t cap, int8_t *__restrict__ Xq,
+                                                          float *__restrict__ S_x, int32_t *__restrict__ out_idx,
+                                                          int32_t *__restrict__ n_out, uint16_t *__restrict__ Xo,
+                                                          int32_t *status) {
+  constexpr int R = 256 / G;
+  extern __shared__ int32_t s_dyn[];  // cap entries of the index list
+  __shared__ int32_t s_scan[9];
+  __shared__ uint32_t red[8];
+  const int tid = threadIdx.x;
+  const int64_t words = (K + 31) >> 5;
+  const int32_t total = build_outlier_list(bitmap, words, cap, s_dyn, s_scan);
+  const int32_t nuse = total < cap ? total : cap;
+  if (blockIdx.x == 0) {
+    for (int j = tid; j < nuse; j += blockDim.x) out_idx[j] = s_dyn[j];
+    if (tid == 0) {
+      *n_out = total;
+      if (total > cap) record_error(status, W8A8_ERR_OUTLIER_OVERFLOW);
+    }
+  }
+
+  const int g = tid / G, t = tid % G;
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * R + g;
+  const bool row_ok = m < M;
+  const int64_t chunks = K >> 3;
+  const uint16_t *xrow = X + m * ldx;
+  uint4 v[VPT];
+  uint32_t amax = 0;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int64_t c = t + static_cast<int64_t>(j) * G;
+    v[j] = make_uint4(0, 0, 0, 0);
+    if (row_ok && c < chunks) {
+      v[j] = __ldcs(reinterpret_cast<const uint4 *>(xrow) + c);
+      // zero the outlier columns of this 8-column chunk
+      const uint32_t mask8 = (__ldg(bitmap + ((c * 8) >> 5)) >> ((c * 8) & 31)) & 0xFFu;
+      if (mask8) {
+        uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          if (mask8 & (1u << (2 * h))) w[h] &= 0xFFFF0000u;
+          if (mask8 & (2u << (2 * h))) w[h] &= 0x0000FFFFu;
+        }
+        v[j] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        amax = max(amax, w[h] & 0x7FFFu);
+        amax = max(amax, (w[h] >> 16) & 0x7FFFu);
+      }
+    }
+  }
+  amax = __reduce_max_sync(0xFFFFFFFFu, amax);
+  if (G > 32) {
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < G / 32; ++w) amax = max(amax, red[w]);
+  }
+  if (!row_ok) return;
+  const float a = __uint_as_float(amax << 16);
+  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+  if (t == 0) S_x[m] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+  int8_t *qrow = Xq + m * K;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int64_t c = t + static_cast<int64_t>(j) * G;
+    if (c < chunks) {
+      const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      int q[8];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        q[2 * h] = min(max(rne_clamped(__fmul_rn(bf16_lo(w[h]), r)), -127), 127);
+        q[2 * h + 1] = min(max(rne_clamped(__fmul_rn(bf16_hi(w[h]), r)), -127), 127);
+      }
+      reinterpret_cast<uint2 *>(qrow)[c] = make_uint2(pack_i8x4(q[0], q[1], q[2], q[3]), pack_i8x4(q[4], q[5], q[6], q[7]));
+    }
+  }
+  // gather this row's outlier values (the row is hot in L1/L2)
+  for (int j = t; j < nuse; j += G) Xo[m * cap + j] = __ldg(xrow + s_dyn[j]);
+}
+
+template <int G, int VPT>
+cudaError_t launch_rows_t(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *bitmap,
+                          int32_t cap, int8_t *Xq, float *S_x, int32_t *idx, int32_t *n_out, uint16_t *Xo,
+                          int32_t *status, cudaStream_t s) {
+  constexpr int R = 256 / G;
+  const size_t smem = static_cast<size_t>(cap > 0 ? cap : 1) * sizeof(int32_t);
+  auto kern = outlier_row_kernel<G, VPT>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  const unsigned blocks = static_cast<unsigned>((M + R - 1) / R);
+  kern<<<blocks, 256, smem, s>>>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t outlier_workspace_bytes(int64_t K) { return static_cast<size_t>(((K + 31) / 32) * 4); }
+
+cudaError_t launch_outlier_split(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, float threshold, int32_t cap,
+                                 int8_t *Xq, float *S_x, int32_t *idx, int32_t *n_out, uint16_t *Xo, void *workspace,
+                                 int32_t *status, cudaStream_t s) {
+  uint32_t *bitmap = static_cast<uint32_t *>(workspace);
+  cudaError_t e = cudaMemsetAsync(bitmap, 0, outlier_workspace_bytes(K), s);
+  if (e != cudaSuccess) return e;
+  const int64_t groups = K / 8;
+  const dim3 grid1(static_cast<unsigned>((groups + 255) / 256), static_cast<unsigned>((M + kRowsPerThread - 1) / kRowsPerThread));
+  outlier_colflag_kernel<<<grid1, 256, 0, s>>>(X, M, K, ldx, threshold, bitmap);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t chunks = K / 8;
+  if (chunks <= 32 * 4) return launch_rows_t<32, 4>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
+  if (chunks <= 32 * 8) return launch_rows_t<32, 8>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
+  if (chunks <= 32 * 16) return launch_rows_t<32, 16>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
+  if (chunks <= 256 * 4) return launch_rows_t<256, 4>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
+  if (chunks <= 256 * 8) return launch_rows_t<256, 8>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
+  if (chunks <= 256 * 16) return launch_rows_t<256, 16>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
+  return launch_rows_t<256, 32>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
+}
+
+}  // namespace w8a8

@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(256) quant_per_tensor_kernel(const uint16_t *_
                                                                const float *__restrict__ r_ptr,
                                                                const int32_t *__restrict__ Z_ptr,
                                                                int8_t *__restrict__ Xq) {
+  pdl_launch_dependents();  // a decode GEMM launched after this one may start streaming weights
   const float r = *r_ptr;
   const int z = *Z_ptr;
   const int64_t cpr = K >> 3;  // chunks per row

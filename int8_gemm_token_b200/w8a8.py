@@ -157,11 +157,21 @@ def w8a8_gemm_workspace_size(M: int, N: int, K: int) -> int:
     return int(lib().w8a8_gemm_workspace_size(M, N, K))
 
 
+def new_workspace(M: int, N: int, K: int, device=None) -> torch.Tensor | None:
+    """A zero-filled workspace for w8a8_gemm_dequant / w8a8_linear_static of
+    this shape (None when the shape needs none). Calls that complete leave it
+    zero-filled, so one workspace serves every later call on the same stream."""
+    n = w8a8_gemm_workspace_size(M, N, K)
+    if n == 0:
+        return None
+    return torch.zeros((n,), dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
 def _workspace(n: int, dev, ws):
     if n == 0:
         return None, 0
     if ws is None:
-        ws = torch.empty((n,), dtype=torch.uint8, device=dev)
+        ws = torch.zeros((n,), dtype=torch.uint8, device=dev)
     return ws, ws.numel() * ws.element_size()
 
 

@@ -192,3 +192,62 @@ def test_bounded_wait_reports_timeout_and_device_stays_usable():
     X = synth.activations(np.random.default_rng(0), 4, 64)
     Xq, S = W.w8a8_quant_per_token(dev_bf16(X))
     assert_same(host(Xq), oracle.quant_per_token(X)[0], "Xq after timeout")
+
+
+# ------------------------------------------------------------ decode kernel (M <= 32)
+def split_k_region_bytes(N):
+    """Leading workspace bytes of the M <= 32 kernel that every completed call
+    leaves zeroed: tile counters (ceil(N/128) x 4 bytes rounded up to 256) and
+    partial sums (ceil(N/128) x 16 KiB), the layout include/w8a8.h documents."""
+    tiles = -(-N // 128)
+    return ((tiles * 4 + 255) // 256) * 256 + tiles * 16384
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (5, 300, 400), (16, 4096, 4096), (17, 520, 1024),
+                                   (32, 11008, 4096), (3, 40, 16), (32, 4096, 11008), (32, 22016, 4096),
+                                   (32, 131072, 512), (16, 131072, 256)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.int32])
+def test_decode_gemm_int8_input_bit_exact(M, N, K, out_dtype):
+    """Small-M GEMM (stream-K split over the weight) with per-token scales."""
+    X, Wf, b = _rand_case(M, N, K, 7 * M + N + K)
+    rq, rS = oracle.quant_per_token(X)
+    rwq, rws, rwc = oracle.quant_weight_per_channel(Wf)
+    ws = W.new_workspace(M, N, K)
+    out = W.w8a8_gemm_dequant(dev(rq), dev(rS), dev(rwq), dev(rws), bias=dev(b), out_dtype=out_dtype, workspace=ws)
+    acc = oracle.gemm_i64(rq, rwq)
+    if out_dtype == torch.int32:
+        assert_same(host(out), acc.astype(np.int32), "acc")
+    else:
+        assert_same(host_bf16(out), oracle.f32_to_bf16(oracle.epilogue(acc, rS, rws, bias=b)), "out")
+    assert int(ws[:split_k_region_bytes(N)].count_nonzero()) == 0, "workspace must be left zeroed"
+
+
+@pytest.mark.parametrize("M,N,K,ld_pad", [(3, 200, 400, 8), (32, 384, 2048, 0), (9, 12288, 4096, 0),
+                                          (32, 22016, 4096, 0), (32, 4096, 11008, 0), (32, 131072, 512, 0),
+                                          (12, 65536, 1024, 24)])
+def test_decode_fused_static_ragged_and_block_shapes(M, N, K, ld_pad):
+    case = synth.decode_static(M=M, N=N, K=K, seed=M + N)
+    S, r, Z = W.w8a8_calibrate_static(dev_bf16(case.Xcal))
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(case.W))
+    bias = synth.bias(np.random.default_rng(1), N)
+    Xd = dev_bf16(np.pad(case.X, ((0, 0), (0, ld_pad))))[:, :K]
+    ws = W.new_workspace(M, N, K)
+    outs = [W.w8a8_linear_static(Xd, S, r, Z, Wq, s_w, cs, bias=dev(bias), workspace=ws) for _ in range(2)]
+    rS, rr, rZ = oracle.calibrate_static(case.Xcal)
+    rwq, rws, rwc = oracle.quant_weight_per_channel(case.W)
+    _, _, y = oracle.linear_decode(case.X, rr, rZ, rS, rwq, rws, rwc, bias=bias)
+    for o in outs:  # the second call reuses the workspace the first one left zeroed
+        assert_same(host_bf16(o), oracle.f32_to_bf16(y), "out")
+    assert int(ws[:split_k_region_bytes(N)].count_nonzero()) == 0
+
+
+def test_decode_fp32_output_and_zero_point():
+    M, N, K = 7, 1000, 512
+    case = synth.decode_static(M=M, N=N, K=K, seed=21)
+    S, r, Z = W.w8a8_calibrate_static(dev_bf16(case.Xcal))
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(case.W))
+    out = W.w8a8_linear_static(dev_bf16(case.X), S, r, Z, Wq, s_w, cs, out_dtype=torch.float32)
+    rS, rr, rZ = oracle.calibrate_static(case.Xcal)
+    rwq, rws, rwc = oracle.quant_weight_per_channel(case.W)
+    _, _, y = oracle.linear_decode(case.X, rr, rZ, rS, rwq, rws, rwc)
+    assert_same(host(out), y, "out")
