@@ -193,6 +193,33 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
                                size_t workspace_bytes, void *stream);
 
 /*
+ * w8a8_linear_static without a workspace argument: the same computation and
+ * result as w8a8_linear_static (same arguments, same checks), for callers
+ * that cannot allocate device memory when they run a Decode step -- a CUDA
+ * graph being captured (cudaMalloc is not a stream operation and breaks the
+ * capture), a plug-in inside a runtime that owns all device memory, or a
+ * latency-critical step that cannot take an allocation's implicit device
+ * synchronization. No counterpart on the pages: this is a deployment entry
+ * point of this library.
+ * The scratch (tile counters, partial sums, quantized activation) is one
+ * fixed device array inside the library, 4,719,616 bytes, held by every GPU
+ * that loads the library until the process exits. It serves M <= 32,
+ * N <= 32768 and K <= 16384; larger shapes return W8A8_ERR_UNSUPPORTED_SHAPE
+ * without launching anything. The call allocates nothing: it clears the part
+ * of the array that must start at zero with cudaMemsetAsync on `stream`,
+ * then launches the same kernels as w8a8_linear_static.
+ * The first call on a device also sets up that device (looks up the array's
+ * device address and zero-fills it once, synchronously): make that first
+ * call before any stream capture. All calls on a device share the one array,
+ * which keeps the last call's contents, so calls that overlap on the GPU
+ * (different streams, or concurrent graphs) race: serialize them.
+ */
+w8a8_status w8a8_linear_static_noalloc(const void *X, int64_t M, int64_t K, int64_t ldx, const float *S,
+                                       const float *r, const int32_t *Z, const int8_t *Wq,
+                                       const float *s_w, const int32_t *colsum, const float *bias,
+                                       int64_t N, void *out, w8a8_dtype out_dtype, void *stream);
+
+/*
  * LLM.int8() outlier split with vector-wise row quantization.
  * Source: LLM.int8() summary, architecture figure: 16-bit decomposition step
  * (1) (pick the columns of X whose magnitude exceeds the threshold, with the

@@ -59,6 +59,18 @@ w8a8_status device_info(DeviceInfo **out) {
   return W8A8_OK;
 }
 
+}  // namespace
+
+w8a8_status current_device_info(int *sm_count, int32_t **status_word) {
+  DeviceInfo *d;
+  if (w8a8_status s = device_info(&d)) return s;
+  *sm_count = d->sm_count;
+  *status_word = d->status;
+  return W8A8_OK;
+}
+
+namespace {
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 

@@ -70,6 +70,10 @@ cudaError_t launch_outlier_split(const uint16_t *X, int64_t M, int64_t K, int64_
                                  int32_t *status, cudaStream_t s);
 size_t outlier_workspace_bytes(int64_t K);
 
+// Per-device set-up of the C ABI (done once per device): SM count and the
+// device address of the device status word.
+w8a8_status current_device_info(int *sm_count, int32_t **status_word);
+
 // 2-D tensor map (driver entry point resolved once per process): inner and
 // outer extents in elements, row stride in bytes, box in elements; swizzle128
 // selects the 128-byte swizzle (box inner extent must then be 128 bytes).

@@ -44,6 +44,7 @@ _SIGNATURES = {
     "w8a8_gemm_dequant": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I32, _P, _SZ, _P]),
     "w8a8_gemm_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "w8a8_linear_static": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _SZ, _P]),
+    "w8a8_linear_static_noalloc": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P]),
     "int8_outlier_split": (_I32, [_P, _I64, _I64, _I64, _F, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "int8_outlier_split_workspace_size": (_SZ, [_I64]),
     "int8_mixed_decomp_gemm": (_I32, [_P, _P, _P, _P, _P, _I32, _P, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _I32, _P]),
@@ -203,6 +204,19 @@ def w8a8_linear_static(X, S, r, Z, Wq, s_w, colsum, bias=None, out=None, out_dty
     _check("w8a8_linear_static", lib().w8a8_linear_static(
         _ptr(X), M, K, _ld(X), _ptr(S), _ptr(r), _ptr(Z), _ptr(Wq), _ptr(s_w), _ptr(colsum),
         _ptr(bias), N, _ptr(out), _dt(out.dtype), _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def w8a8_linear_static_noalloc(X, S, r, Z, Wq, s_w, colsum, bias=None, out=None, out_dtype=torch.bfloat16,
+                               stream=None):
+    """w8a8_linear_static with the library's own fixed scratch instead of a
+    caller workspace (M <= 32, N <= 32768, K <= 16384)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    out = torch.empty((M, N), dtype=out_dtype, device=X.device) if out is None else out
+    _check("w8a8_linear_static_noalloc", lib().w8a8_linear_static_noalloc(
+        _ptr(X), M, K, _ld(X), _ptr(S), _ptr(r), _ptr(Z), _ptr(Wq), _ptr(s_w), _ptr(colsum), _ptr(bias), N,
+        _ptr(out), _dt(out.dtype), _stream(stream)))
     return out
 
 

@@ -88,6 +88,10 @@ def test_other_entry_points_host_checks(L):
                                     8, 8, 64, GOOD, 2, None) == 4  # int32 output not offered here
     assert L.int8_mixed_decomp_gemm(GOOD, GOOD, GOOD, GOOD, GOOD, 5000, GOOD, GOOD, GOOD, 8, None,
                                     8, 8, 64, GOOD, 0, None) == 1
+    # X, M, K, ldx, S, r, Z, Wq, s_w, colsum, bias, N, out, dt, stream
+    assert L.w8a8_linear_static_noalloc(GOOD, 33, 64, 64, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, None, 8, GOOD, 0, None) == 3
+    assert L.w8a8_linear_static_noalloc(GOOD, 4, 16400, 16400, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, None, 8, GOOD, 0, None) == 3
+    assert L.w8a8_linear_static_noalloc(GOOD, 4, 64, 64, GOOD, GOOD, None, GOOD, GOOD, GOOD, None, 8, GOOD, 0, None) == 1
     assert L.w8a8_debug_wait_timeout_selftest(10, None) == 1
     st = ctypes.c_int32(0)
     assert L.w8a8_check_device_error(None, None) == 1
