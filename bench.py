@@ -15,8 +15,11 @@ is bracketed by a barrier and the slowest rank's time is reported.
 --impl reference times the CPU oracle (a plain C implementation, OpenMP over
 rows) on a bounded sample of the same workload.
 
-The JSON line also carries a Decode measurement (fused static-quant linear,
-32 tokens x 4096 -> 11008, HBM-bound) under "decode".
+The JSON line also carries the other rows of the path, each measured on its
+own workload: "decode" (fused static-quant Decode linear, 1-32 tokens x 4096
+-> 11008 / 4096, HBM-bound, CUDA-graph timed), "llm_int8" (outlier split and
+mixed-decomposition GEMM at 4096 x 8192 x 8192) and "pdmix_block" (four
+Llama-7B-like linears: a 4096-token Prefill pass and 64 Decode steps).
 """
 from __future__ import annotations
 
@@ -88,7 +91,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.005)
 
     def __enter__(self):
         if self.nv is not None:
@@ -264,12 +267,16 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms,
                "steps": e2e_steps}
 
-    # ---------------------------------------------------------------- decode
-    decode = None
-    if not args.no_decode:
-        decode = bench_decode(args, dev, rank, peaks, max_over_ranks, barrier)
-
     del sets
+    torch.cuda.empty_cache()
+    # ---------------------------------------------------------------- the other rows of the path
+    decode = llm = block = None
+    if not args.no_decode:
+        decode = bench_decode(args, dev, rank, peaks)
+    if not args.no_llm_int8:
+        llm = bench_llm_int8(args, dev, rank, peaks, int8_peak)
+    if not args.no_block:
+        block = bench_block(args, dev, rank, peaks, int8_peak)
     line = None
     if rank == 0:
         cpu = None
@@ -295,6 +302,8 @@ def run_ours(args, world, rank, local):
                       "C_s_over_C_g": quant_ms / gemm_ms},
             "gemm_ms": gemm_ms,
             "decode": decode,
+            "llm_int8": llm,
+            "pdmix_block": block,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 2 * args.steps,
@@ -304,51 +313,178 @@ def run_ours(args, world, rank, local):
     return 0
 
 
-def bench_decode(args, dev, rank, peaks, max_over_ranks, barrier):
-    """Fused static-quant Decode linear, 32 x 4096 -> 11008, rotating 6 weights (> L2)."""
+def graph_time_us(fn, n_calls, reps=10):
+    """Per-call device time of fn(i), i < n_calls, captured once in a CUDA
+    graph and replayed `reps` times between two events (no host overhead)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for i in range(min(3, n_calls)):
+            fn(i)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n_calls):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) * 1e3 / (reps * n_calls)
+
+
+def bench_decode(args, dev, rank, peaks):
+    """Fused static-quant Decode linear (PDMIX decode: per-tensor static
+    asymmetric quant + INT8 GEMM + zero-point corrected epilogue), for the
+    token counts and weight shapes of the Decode workload, weights rotated so
+    every call streams its weight from HBM; graph-timed."""
     import torch
 
     from int8_gemm_token_b200 import synth
     from int8_gemm_token_b200 import w8a8 as W
-    n_w = 6
-    case = synth.decode_static(M=DEC_M, N=DEC_N, K=DEC_K, seed=rank)
-    X = torch.from_numpy(case.X.view(np.int16)).view(torch.bfloat16).to(dev)
-    S, r, Z = W.w8a8_calibrate_static(torch.from_numpy(case.Xcal.view(np.int16)).view(torch.bfloat16).to(dev))
-    ws = []
-    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(torch.from_numpy(case.W).to(dev))
-    for i in range(n_w):
-        ws.append((Wq.clone(), s_w.clone(), cs.clone(), torch.empty((DEC_M, DEC_N), dtype=torch.bfloat16, device=dev)))
-    work = W.new_workspace(DEC_M, DEC_N, DEC_K, device=dev)
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    rows = []
+    for N in (11008, 4096):
+        case = synth.decode_static(M=32, N=N, K=DEC_K, seed=rank)
+        S, r, Z = W.w8a8_calibrate_static(bf(case.Xcal))
+        Wq, s_w, cs = W.w8a8_quant_weight_per_channel(torch.from_numpy(case.W).to(dev))
+        n_w = max(3, int(600e6 // (N * DEC_K)) + 1)
+        ws = [(Wq.clone(), s_w.clone(), cs.clone()) for _ in range(n_w)]
+        Xall = bf(case.X)
+        for M in (32, 16, 4, 1):
+            X = Xall[:M].contiguous()
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            work = W.new_workspace(M, N, DEC_K, device=dev)
+            us = graph_time_us(lambda i: W.w8a8_linear_static(X, S, r, Z, *ws[i % n_w], out=out, workspace=work), 2 * n_w)
+            nbytes = N * DEC_K + 8.0 * N + 2.0 * M * DEC_K + 2.0 * M * N
+            gbs = nbytes / (us * 1e-6) / 1e9
+            rows.append({"M": M, "K": DEC_K, "N": N, "us": us, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]})
+        del ws
+    # static quant alone vs GEMM alone (the C_s / C_g of the PDMIX cost model) at the largest shape
+    return {"workload": "decode: fused static-quant W8A8 linear (quant kernel + PDL-overlapped stream-K GEMM), "
+                        f"rotating weights > L2, CUDA-graph timed", "rows": rows,
+            "unit": "GB/s", "peak": peaks["hbm_gbs"], "algorithmic_bytes": "N*K + 8N + 2MK + 2MN per call"}
+
+
+def bench_llm_int8(args, dev, rank, peaks, int8_peak):
+    """LLM.int8() mode at 4096 x 8192 x 8192: outlier split + mixed GEMM."""
+    import torch
+
+    from int8_gemm_token_b200 import synth
+    from int8_gemm_token_b200 import w8a8 as W
+    case = synth.llm_int8(seed=rank)
+    bf = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)
+    X, Wd = bf(case.X), bf(case.W)
+    Mq, Kq = case.X.shape
+    Nq = case.W.shape[1]
+    cap = 64
+    Wq, s_w, _ = W.w8a8_quant_weight_per_channel(Wd)
+    Xq = torch.empty((Mq, Kq), dtype=torch.int8, device=dev)
+    S = torch.empty((Mq,), dtype=torch.float32, device=dev)
+    idx = torch.empty((cap,), dtype=torch.int32, device=dev)
+    n_out = torch.empty((1,), dtype=torch.int32, device=dev)
+    Xo = torch.empty((Mq, cap), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((Mq, Nq), dtype=torch.bfloat16, device=dev)
+    wsb = torch.zeros((W.lib().int8_outlier_split_workspace_size(Kq),), dtype=torch.uint8, device=dev)
+    split = lambda i: W.int8_outlier_split(X, case.threshold, cap, Xq=Xq, S_x=S, idx=idx, n_out=n_out, Xo=Xo, workspace=wsb)
+    gemm = lambda i: W.int8_mixed_decomp_gemm(Xq, S, Xo, idx, n_out, cap, Wq, s_w, Wd, out=out)
+    split_us = graph_time_us(split, 4)
+    gemm_us = graph_time_us(gemm, 4)
+    split_bytes = 2.0 * Mq * Kq + Mq * Kq + 4.0 * Mq + 2.0 * Mq * int(n_out.item())
+    ops = 2.0 * Mq * Nq * Kq
+    assert W.w8a8_check_device_error() == 0
+    return {"workload": f"LLM.int8() X [{Mq} x {Kq}] ({int(n_out.item())} outlier columns), W bf16 [{Kq} x {Nq}], threshold 6.0",
+            "split_us": split_us, "split_GB/s": split_bytes / (split_us * 1e-6) / 1e9,
+            "split_frac_hbm": split_bytes / (split_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+            "split_algorithmic_bytes": split_bytes,
+            "mixed_gemm_us": gemm_us, "mixed_gemm_TOPS": ops / (gemm_us * 1e-6) / 1e12,
+            "mixed_gemm_frac_int8": ops / (gemm_us * 1e-6) / 1e12 / int8_peak}
+
+
+def bench_block(args, dev, rank, peaks, int8_peak):
+    """PDMIX block sequence (Llama-7B-like linears): one Prefill pass of 4096
+    tokens (per-token quant + GEMM per linear) and 64 Decode steps of 32 tokens
+    (fused static-quant linear per linear), one INT8 weight per linear shared
+    by both phases; decode steps captured in one CUDA graph."""
+    import torch
+
+    from int8_gemm_token_b200 import synth
+    from int8_gemm_token_b200 import w8a8 as W
+    bf = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)
+    lin = synth.pdmix_block(seed=rank)
+    layers = []
+    for L_ in lin:
+        Wq, s_w, cs = W.w8a8_quant_weight_per_channel(torch.from_numpy(L_.weight()).to(dev))
+        S, r, Z = W.w8a8_calibrate_static(bf(L_.calibration()))
+        Xp = bf(L_.prefill_input(4096))
+        dec = torch.stack([bf(L_.decode_input(step, 32)) for step in range(64)])
+        layers.append(dict(K=L_.K, N=L_.N, Wq=Wq, s_w=s_w, cs=cs, S=S, r=r, Z=Z, Xp=Xp, dec=dec,
+                           Xq=torch.empty((4096, L_.K), dtype=torch.int8, device=dev),
+                           Sx=torch.empty((4096,), dtype=torch.float32, device=dev),
+                           outp=torch.empty((4096, L_.N), dtype=torch.bfloat16, device=dev),
+                           outd=torch.empty((32, L_.N), dtype=torch.bfloat16, device=dev),
+                           work=W.new_workspace(32, L_.N, L_.K, device=dev)))
     stream = torch.cuda.current_stream()
-    steps = max(args.steps, 20)
-    for i in range(max(args.warmup, 3)):
-        q, s, c, o = ws[i % n_w]
-        W.w8a8_linear_static(X, S, r, Z, q, s, c, out=o, workspace=work, stream=stream)
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    barrier()
-    for i in range(steps):
-        q, s, c, o = ws[i % n_w]
-        ev[i][0].record(stream)
-        W.w8a8_linear_static(X, S, r, Z, q, s, c, out=o, workspace=work, stream=stream)
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev))
-    nbytes = DEC_N * DEC_K + 8.0 * DEC_N + 2.0 * DEC_M * DEC_K + 2.0 * DEC_M * DEC_N
-    gbs = nbytes / (ms * 1e-3) / 1e9
-    return {"workload": f"decode fused static-quant linear M={DEC_M} K={DEC_K} N={DEC_N}, {n_w} rotating weights",
-            "us_per_layer": ms * 1e3, "achieved": gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
-            "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": nbytes}
+    # prefill: events around each kernel, a few repetitions
+    q_ms = g_ms = 0.0
+    reps = 5
+    for rep in range(reps + 2):
+        evs = []
+        for Ly in layers:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            W.w8a8_quant_per_token(Ly["Xp"], Xq=Ly["Xq"], S_x=Ly["Sx"])
+            e[1].record(stream)
+            W.w8a8_gemm_dequant(Ly["Xq"], Ly["Sx"], Ly["Wq"], Ly["s_w"], out=Ly["outp"])
+            e[2].record(stream)
+            evs.append(e)
+        torch.cuda.synchronize()
+        if rep >= 2:
+            q_ms += sum(e[0].elapsed_time(e[1]) for e in evs) / reps
+            g_ms += sum(e[1].elapsed_time(e[2]) for e in evs) / reps
+    prefill_ops = sum(2.0 * 4096 * Ly["K"] * Ly["N"] for Ly in layers)
+
+    def decode_all(step):
+        for Ly in layers:
+            W.w8a8_linear_static(Ly["dec"][step], Ly["S"], Ly["r"], Ly["Z"], Ly["Wq"], Ly["s_w"], Ly["cs"],
+                                 out=Ly["outd"], workspace=Ly["work"])
+    step_us = graph_time_us(decode_all, 64, reps=3)
+    w_bytes = sum(Ly["K"] * Ly["N"] for Ly in layers)
+    # the PDMIX cost model: static quant alone vs the decode GEMM alone, per step
+    dq_us = graph_time_us(lambda i: [W.w8a8_quant_per_tensor(Ly["dec"][i % 64], Ly["r"], Ly["Z"], Xq=Ly["Xq"][:32]) for Ly in layers], 16)
+    assert W.w8a8_check_device_error() == 0
+    return {"workload": "PDMIX block: QKV 4096->12288, O 4096->4096, gate+up 4096->22016, down 11008->4096; "
+                        "prefill 4096 tokens, then 64 decode steps x 32 tokens",
+            "prefill_us": (q_ms + g_ms) * 1e3, "prefill_TOPS": prefill_ops / ((q_ms + g_ms) * 1e-3) / 1e12,
+            "prefill_gemm_frac_int8": prefill_ops / (g_ms * 1e-3) / 1e12 / int8_peak,
+            "prefill_C_s_over_C_g": q_ms / g_ms,
+            "decode_total_us": 64 * step_us, "decode_step_us": step_us,
+            "decode_weight_GB/s": w_bytes / (step_us * 1e-6) / 1e9,
+            "decode_frac_hbm": w_bytes / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+            "decode_static_quant_us_per_step": dq_us,
+            "decode_C_s_over_C_g": dq_us / max(step_us - dq_us, 1e-9)}
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-llm-int8", action="store_true")
+    ap.add_argument("--no-block", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=16)

@@ -225,6 +225,78 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- CTA pairs
+// Rank of this CTA in its cluster.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address, in the cluster's shared window, of the same shared-memory offset in
+// CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_addr(p)), "r"(rank));
+  return out;
+}
+
+// All threads of all CTAs of the cluster (call it from every thread).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on an mbarrier given by its cluster-window address (another CTA's).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// 2-D TMA load for a CTA pair: lands in this CTA's shared memory and signals
+// the mbarrier at `bar_cluster_addr` (the pair leader's), no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_cluster_addr, void *dst,
+                                                 int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T over the pair
+// (M = 256: each CTA holds 128 rows of A and of D; B's N rows are split
+// between the two CTAs' shared memory). Issued by one thread of the leader.
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the mbarrier at `bar_cluster_addr` (any CTA of the pair) when
+// the pair MMAs issued so far by this thread have completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar_cluster_addr) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar_cluster_addr)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- numerics
 // bf16 <-> fp32 on raw bits.
 __device__ __forceinline__ float bf16_lo(uint32_t two) { return __uint_as_float(two << 16); }
@@ -241,6 +313,62 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ int rne_clamped(float p) {
   int t = __float2int_rn(p);
   return min(max(t, -1024), 1024);
+}
+
+// Round to nearest even into int32 (out-of-range values saturate).
+__device__ __forceinline__ int rne_s32(float p) {
+  int r;
+  asm("cvt.rni.s32.f32 %0, %1;" : "=r"(r) : "f"(p));
+  return r;
+}
+
+__device__ __forceinline__ int add_sat_s32(int a, int b) {
+  int r;
+  asm("add.sat.s32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Four int32 saturated to [-128, 127] and packed, a in the lowest byte.
+__device__ __forceinline__ uint32_t pack_sat_s8x4(int a, int b, int c, int d) {
+  uint32_t hi, out;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(d), "r"(c));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(out) : "r"(b), "r"(a), "r"(hi));
+  return out;
+}
+
+// Symmetric codes of the 8 bf16 values in one uint4: clamp(rne(x * r), -127, 127). With r = 127/absmax every |x * r|
+// is at most 127 * (1 + 2^-23), so saturating to [-128, 127] equals that clamp.
+__device__ __forceinline__ uint2 quant8_sym_sat(const uint4 &v, float r) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  int q[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    q[2 * i] = rne_s32(__fmul_rn(bf16_lo(w[i]), r));
+    q[2 * i + 1] = rne_s32(__fmul_rn(bf16_hi(w[i]), r));
+  }
+  return make_uint2(pack_sat_s8x4(q[0], q[1], q[2], q[3]), pack_sat_s8x4(q[4], q[5], q[6], q[7]));
+}
+
+// Static asymmetric codes: clamp(rne(x * r) + Z, -128, 127) (saturating add,
+// so huge inputs cannot wrap).
+__device__ __forceinline__ uint2 quant8_asym_sat(const uint4 &v, float r, int z) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  int q[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    q[2 * i] = add_sat_s32(rne_s32(__fmul_rn(bf16_lo(w[i]), r)), z);
+    q[2 * i + 1] = add_sat_s32(rne_s32(__fmul_rn(bf16_hi(w[i]), r)), z);
+  }
+  return make_uint2(pack_sat_s8x4(q[0], q[1], q[2], q[3]), pack_sat_s8x4(q[4], q[5], q[6], q[7]));
+}
+
+// Running per-halfword maximum of bf16 magnitudes (two values per word).
+__device__ __forceinline__ uint32_t absmax2_u4(const uint4 &v, uint32_t m2) {
+  m2 = __vmaxu2(m2, v.x & 0x7FFF7FFFu);
+  m2 = __vmaxu2(m2, v.y & 0x7FFF7FFFu);
+  m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
+  m2 = __vmaxu2(m2, v.w & 0x7FFF7FFFu);
+  return m2;
 }
 
 __device__ __forceinline__ uint32_t pack_i8x4(int a, int b, int c, int d) {

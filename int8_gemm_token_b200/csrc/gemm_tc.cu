@@ -356,6 +356,243 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- CTA pairs
+// The same GEMM with 256 x 256 output tiles computed by a cluster of two CTAs
+// (tcgen05.mma cta_group::2): each CTA of the pair loads its own 128 rows of
+// Xq and its own 128 rows of Wq per k-block (32 KiB), the leader issues the
+// pair MMA (M = 256, N = 256), and each CTA holds its 128 rows of the
+// accumulator in its own TMEM. Per SM this moves 2/3 of the operand bytes of a
+// single-CTA 128 x 256 tile for the same tensor work.
+//   leader (rank 0): full barriers (expect_tx for both CTAs' loads, which
+//                    complete_tx on the leader's barrier), MMA issue, commits
+//                    to the empty / accumulator-full barriers of both CTAs,
+//                    accumulator-empty barrier counting both CTAs' epilogues;
+//   both:            TMA loads into their own shared memory, epilogue.
+template <int STAGES, bool MIXED>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_i8_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       int64_t M, int64_t N, int64_t K, const __grid_constant__ EpilogueArgs ep,
+                       int32_t *status, uint64_t limit_ns) {
+  constexpr int kHalf = 128;                 // rows of A and of B per CTA
+  constexpr int kStageA2 = kHalf * kBK;      // 16 KiB
+  constexpr int kStageB2 = kHalf * kBK;      // 16 KiB
+  constexpr int kTileM = 256, kTileN = 256;  // pair tile
+  constexpr uint32_t kTmemCols = 512;        // two 256-column accumulators
+  constexpr uint32_t kIdesc = idesc_i8(kTileM, kTileN);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = base;
+  uint8_t *sB = base + STAGES * kStageA2;
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sB + STAGES * kStageB2);
+  uint64_t *empty_bar = full_bar + STAGES;
+  uint64_t *tfull_bar = empty_bar + STAGES;
+  uint64_t *tempty_bar = tfull_bar + 2;
+  uint64_t *drain_bar = tempty_bar + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncwarp();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t num_m = (M + kTileM - 1) / kTileM;
+  const int64_t num_n = (N + kTileN - 1) / kTileN;
+  const int64_t num_tiles = num_m * num_n;
+  const int nkb = static_cast<int>((K + kBK - 1) / kBK);
+  const int64_t cluster_id = blockIdx.x >> 1;
+  const int64_t num_clusters = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+        const int32_t arow = static_cast<int32_t>((tile % num_m) * kTileM + rank * kHalf);
+        const int32_t brow = static_cast<int32_t>((tile / num_m) * kTileN + rank * kHalf);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag, limit_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t leader_full = map_to_rank(&full_bar[stage], 0);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * (kStageA2 + kStageB2));
+          tma_load_2d_pair(&tmA, leader_full, sA + stage * kStageA2, kb * kBK, arow);
+          tma_load_2d_pair(&tmB, leader_full, sB + stage * kStageB2, kb * kBK, brow);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ pair MMA issuer (leader)
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int64_t tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+        if (!mbar_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, limit_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kTileN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&full_bar[stage], phase, abort_flag, limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(sA + stage * kStageA2);
+          const uint32_t b_addr = smem_addr(sB + stage * kStageB2);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_i8_pair(d_tmem, smem_desc_k_sw128(a_addr + 32 * k), smem_desc_k_sw128(b_addr + 32 * k), kIdesc,
+                        (kb | k) != 0 ? 1u : 0u);
+          mma_commit_pair(map_to_rank(&empty_bar[stage], 0));
+          mma_commit_pair(map_to_rank(&empty_bar[stage], 1));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(map_to_rank(&tfull_bar[acc], 0));
+        mma_commit_pair(map_to_rank(&tfull_bar[acc], 1));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+        mma_commit_pair(map_to_rank(drain_bar, 0));
+        mbar_wait_bounded(drain_bar, 0, nullptr, limit_ns / 16 + 1);
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // -------------------------------------------------- epilogue (both CTAs)
+    const int q = warp - kEpiWarp0;
+    const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
+    int32_t nuse = 0;
+    if (MIXED) nuse = min(__ldg(ep.n_out), ep.cap);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t tile = cluster_id; tile < num_tiles; tile += num_clusters) {
+      const bool ready = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag, limit_ns));
+      if (!ready) {
+        if (lane == 0) {
+          record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const int64_t m = (tile % num_m) * kTileM + rank * kHalf + q * 32 + lane;
+      const int64_t nbase = (tile / num_m) * kTileN;
+      float sx = 0.0f;
+      if (m < M) sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : __ldg(ep.S_x);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kTileN);
+#pragma unroll 1
+      for (int c = 0; c < kTileN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, r);
+        tmem_ld_wait();
+        epilogue_chunk<MIXED>(r, m, nbase + c * 32, M, N, sx, z, ep, nuse);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&tempty_bar[acc]);
+        else
+          mbar_arrive_remote(map_to_rank(&tempty_bar[acc], 0));
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the pair still reads its memory or barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+template <int STAGES, bool MIXED>
+cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
+                         const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
+  constexpr size_t kSmem = static_cast<size_t>(STAGES) * 2 * 128 * kBK + 1024 + 256;
+  alignas(64) CUtensorMap tmA, tmB;
+  if (!encode_tmap_2d(&tmA, Xq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                      static_cast<uint64_t>(K), kBK, 128, true))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(&tmB, Wq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                      static_cast<uint64_t>(K), kBK, 128, true))
+    return cudaErrorInvalidValue;
+  auto kern = gemm_i8_tc2_kernel<STAGES, MIXED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  const int64_t pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, M, N, K, ep, status, kWaitLimitNs);
+}
+
 template <int BN, int STAGES, bool MIXED>
 cudaError_t launch_tc_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                         const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
@@ -383,6 +620,11 @@ cudaError_t launch_tc_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N
 cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                            const EpilogueArgs &ep, bool mixed, int num_sms, int32_t *status,
                            cudaStream_t s) {
+  // CTA pairs (256-row tiles) once there are enough rows to fill them
+  if (M >= 256 && num_sms >= 2) {
+    if (mixed) return launch_tc2_t<6, true>(Xq, Wq, M, N, K, ep, num_sms, status, s);
+    return launch_tc2_t<6, false>(Xq, Wq, M, N, K, ep, num_sms, status, s);
+  }
   if (mixed) return launch_tc_t<256, 4, true>(Xq, Wq, M, N, K, ep, num_sms, status, s);
   return launch_tc_t<256, 4, false>(Xq, Wq, M, N, K, ep, num_sms, status, s);
 }

@@ -37,7 +37,8 @@ __global__ void __launch_bounds__(256) outlier_colflag_kernel(const uint16_t *__
   if (g >= groups) return;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kRowsPerThread;
   const int64_t r1 = r0 + kRowsPerThread < M ? r0 + kRowsPerThread : M;
-  uint32_t mx[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // magnitude bits per column
+  // magnitude bits of the 8 columns, two per word (packed unsigned maxima)
+  uint32_t mx0 = 0, mx1 = 0, mx2 = 0, mx3 = 0;
   const uint4 *p = reinterpret_cast<const uint4 *>(X + r0 * ldx) + g;
   const int64_t step = ldx >> 3;
   int64_t r = r0;
@@ -47,29 +48,28 @@ __global__ void __launch_bounds__(256) outlier_colflag_kernel(const uint16_t *__
     for (int i = 0; i < 8; ++i) v[i] = __ldcs(p + i * step);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        mx[2 * j] = max(mx[2 * j], w[j] & 0x7FFFu);
-        mx[2 * j + 1] = max(mx[2 * j + 1], (w[j] >> 16) & 0x7FFFu);
-      }
+      mx0 = __vmaxu2(mx0, v[i].x & 0x7FFF7FFFu);
+      mx1 = __vmaxu2(mx1, v[i].y & 0x7FFF7FFFu);
+      mx2 = __vmaxu2(mx2, v[i].z & 0x7FFF7FFFu);
+      mx3 = __vmaxu2(mx3, v[i].w & 0x7FFF7FFFu);
     }
     p += 8 * step;
   }
   for (; r < r1; ++r) {
     const uint4 v = __ldcs(p);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      mx[2 * j] = max(mx[2 * j], w[j] & 0x7FFFu);
-      mx[2 * j + 1] = max(mx[2 * j + 1], (w[j] >> 16) & 0x7FFFu);
-    }
+    mx0 = __vmaxu2(mx0, v.x & 0x7FFF7FFFu);
+    mx1 = __vmaxu2(mx1, v.y & 0x7FFF7FFFu);
+    mx2 = __vmaxu2(mx2, v.z & 0x7FFF7FFFu);
+    mx3 = __vmaxu2(mx3, v.w & 0x7FFF7FFFu);
     p += step;
   }
+  const uint32_t mw[4] = {mx0, mx1, mx2, mx3};
   uint32_t bits = 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (__uint_as_float(mx[j] << 16) > threshold) bits |= 1u << j;
+  for (int j = 0; j < 4; ++j) {
+    if (__uint_as_float(mw[j] << 16) > threshold) bits |= 1u << (2 * j);
+    if (__uint_as_float(mw[j] & 0xFFFF0000u) > threshold) bits |= 2u << (2 * j);
+  }
   if (bits) atomicOr(bitmap + ((g * 8) >> 5), bits << ((g * 8) & 31));
 }
 
@@ -166,14 +166,10 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
         }
         v[j] = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        amax = max(amax, w[h] & 0x7FFFu);
-        amax = max(amax, (w[h] >> 16) & 0x7FFFu);
-      }
+      amax = absmax2_u4(v[j], amax);
     }
   }
+  amax = max(amax & 0xFFFFu, amax >> 16);
   amax = __reduce_max_sync(0xFFFFFFFFu, amax);
   if (G > 32) {
     if ((tid & 31) == 0) red[tid >> 5] = amax;
@@ -190,16 +186,7 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int64_t c = t + static_cast<int64_t>(j) * G;
-    if (c < chunks) {
-      const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-      int q[8];
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        q[2 * h] = min(max(rne_clamped(__fmul_rn(bf16_lo(w[h]), r)), -127), 127);
-        q[2 * h + 1] = min(max(rne_clamped(__fmul_rn(bf16_hi(w[h]), r)), -127), 127);
-      }
-      reinterpret_cast<uint2 *>(qrow)[c] = make_uint2(pack_i8x4(q[0], q[1], q[2], q[3]), pack_i8x4(q[4], q[5], q[6], q[7]));
-    }
+    if (c < chunks) reinterpret_cast<uint2 *>(qrow)[c] = quant8_sym_sat(v[j], r);
   }
   // gather this row's outlier values (the row is hot in L1/L2)
   for (int j = t; j < nuse; j += G) Xo[m * cap + j] = __ldg(xrow + s_dyn[j]);

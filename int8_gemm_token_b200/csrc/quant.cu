@@ -18,47 +18,17 @@ namespace w8a8 {
 // ------------------------------------------------------------------ helpers
 // |x| of bf16 values compared on their bit patterns: for finite values the
 // magnitude bits order exactly like the magnitudes.
-__device__ __forceinline__ uint32_t absmax_bits_u4(const uint4 &v, uint32_t m) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    m = max(m, w[i] & 0x7FFFu);
-    m = max(m, (w[i] >> 16) & 0x7FFFu);
-  }
-  return m;
-}
-
-__device__ __forceinline__ uint2 quant8_sym(const uint4 &v, float r) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  int q[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    q[2 * i] = min(max(rne_clamped(__fmul_rn(bf16_lo(w[i]), r)), -127), 127);
-    q[2 * i + 1] = min(max(rne_clamped(__fmul_rn(bf16_hi(w[i]), r)), -127), 127);
-  }
-  return make_uint2(pack_i8x4(q[0], q[1], q[2], q[3]), pack_i8x4(q[4], q[5], q[6], q[7]));
-}
-
-__device__ __forceinline__ uint2 quant8_asym(const uint4 &v, float r, int z) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  int q[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    q[2 * i] = min(max(rne_clamped(__fmul_rn(bf16_lo(w[i]), r)) + z, -128), 127);
-    q[2 * i + 1] = min(max(rne_clamped(__fmul_rn(bf16_hi(w[i]), r)) + z, -128), 127);
-  }
-  return make_uint2(pack_i8x4(q[0], q[1], q[2], q[3]), pack_i8x4(q[4], q[5], q[6], q[7]));
-}
-
 // ------------------------------------------------------------ per token
 // G threads per row (32 = one warp, or 256 = the whole block), VPT 16-byte
 // chunks (8 bf16) per thread held in registers, so X is read exactly once.
+// Warp-per-row blocks hold 4 rows, so the rows spread evenly over the SMs.
 template <int G, int VPT>
 __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__restrict__ X,
                                                               int64_t M, int64_t K, int64_t ldx,
                                                               int8_t *__restrict__ Xq,
                                                               float *__restrict__ S_x) {
-  constexpr int R = 256 / G;  // rows per block
+  constexpr int NT = G == 32 ? 128 : 256;  // threads per block
+  constexpr int R = NT / G;                // rows per block
   __shared__ uint32_t red[8];
   const int tid = threadIdx.x;
   const int g = tid / G;  // row slot in this block
@@ -69,17 +39,18 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__
   const uint16_t *xrow = X + m * ldx;
 
   uint4 v[VPT];
-  uint32_t amax = 0;
+  uint32_t m2 = 0;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int64_t c = t + static_cast<int64_t>(j) * G;
     if (row_ok && c < chunks) {
       v[j] = __ldcs(reinterpret_cast<const uint4 *>(xrow) + c);
-      amax = absmax_bits_u4(v[j], amax);
+      m2 = absmax2_u4(v[j], m2);
     } else {
       v[j] = make_uint4(0, 0, 0, 0);
     }
   }
+  uint32_t amax = max(m2 & 0xFFFFu, m2 >> 16);
   amax = __reduce_max_sync(0xFFFFFFFFu, amax);
   if (G > 32) {
     if ((tid & 31) == 0) red[tid >> 5] = amax;
@@ -97,16 +68,17 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int64_t c = t + static_cast<int64_t>(j) * G;
-    if (c < chunks) reinterpret_cast<uint2 *>(qrow)[c] = quant8_sym(v[j], r);
+    if (c < chunks) reinterpret_cast<uint2 *>(qrow)[c] = quant8_sym_sat(v[j], r);
   }
 }
 
 template <int G, int VPT>
 static cudaError_t launch_per_token_t(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                       int8_t *Xq, float *S_x, cudaStream_t s) {
-  constexpr int R = 256 / G;
+  constexpr int NT = G == 32 ? 128 : 256;
+  constexpr int R = NT / G;
   const unsigned blocks = static_cast<unsigned>((M + R - 1) / R);
-  quant_per_token_kernel<G, VPT><<<blocks, 256, 0, s>>>(X, M, K, ldx, Xq, S_x);
+  quant_per_token_kernel<G, VPT><<<blocks, NT, 0, s>>>(X, M, K, ldx, Xq, S_x);
   return cudaGetLastError();
 }
 
@@ -140,7 +112,7 @@ __global__ void __launch_bounds__(256) quant_per_tensor_kernel(const uint16_t *_
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t m = i / cpr, c = i - m * cpr;
     const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(X + m * ldx) + c);
-    reinterpret_cast<uint2 *>(Xq + m * K)[c] = quant8_asym(v, r, z);
+    reinterpret_cast<uint2 *>(Xq + m * K)[c] = quant8_asym_sat(v, r, z);
   }
 }
 

@@ -22,6 +22,7 @@ HEADER = os.path.join(ROOT, "include", "w8a8.h")
 
 OK = 0
 BF16, FP32, I32 = 0, 1, 2
+DECODE_MAX_M = 32  # calls with at most this many tokens take the split-K decode kernel
 STATUS_NAMES = {}
 
 
@@ -187,7 +188,8 @@ def w8a8_gemm_dequant(Xq, S_x, Wq, s_w, colsum=None, Z=None, bias=None, out=None
     if S_x.numel() not in (1, M):
         raise ValueError("S_x holds one scale per row or a single per-tensor scale")
     per_row = 1 if S_x.numel() == M else 0
-    ws, nbytes = _workspace(w8a8_gemm_workspace_size(M, N, K), Xq.device, workspace)
+    # only the decode-shaped kernel (M <= 32) uses a workspace in this call
+    ws, nbytes = _workspace(w8a8_gemm_workspace_size(M, N, K) if M <= DECODE_MAX_M else 0, Xq.device, workspace)
     _check("w8a8_gemm_dequant", lib().w8a8_gemm_dequant(
         _ptr(Xq), _ptr(S_x), per_row, _ptr(Z), _ptr(Wq), _ptr(s_w), _ptr(colsum), _ptr(bias),
         M, N, K, _ptr(out), _dt(out.dtype), _ptr(ws), nbytes, _stream(stream)))
