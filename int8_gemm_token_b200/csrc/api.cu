@@ -291,7 +291,8 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
     // programmatic dependent launch: its weight stream starts while the
     // quantization runs, and it reads the quantized activation after it.
     int8_t *Xq = static_cast<int8_t *>(workspace) + decode_counters_bytes(N) + decode_partials_bytes(N);
-    cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq, d->sm_count, st);
+    cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq, d->sm_count, st,
+                                            /*pdl=*/true);
     if (e != cudaSuccess) return W8A8_ERR_CUDA;
     return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, workspace, true, d->sm_count, d->status, st));
   }

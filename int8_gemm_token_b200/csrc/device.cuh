@@ -225,6 +225,17 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// atomicAdd with release semantics at GPU scope: every write that precedes it
+// (including other threads' writes ordered before it by a barrier) is visible
+// before the addition is.
+__device__ __forceinline__ uint32_t atomic_add_release_gpu(uint32_t *p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 // ---------------------------------------------------------------- CTA pairs
 // Rank of this CTA in its cluster.
 __device__ __forceinline__ uint32_t cluster_rank() {

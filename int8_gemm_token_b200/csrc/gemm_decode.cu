@@ -53,14 +53,16 @@ namespace {
 constexpr int kBK = 128;                 // bytes of K per k-block (one swizzle row)
 constexpr int kTileN = 128;              // weight rows per tile = MMA M = TMEM lanes
 constexpr int kStageW = kTileN * kBK;    // 16 KiB
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4-7 and 8-11 two epilogue sets
 constexpr int kEpiWarp0 = 4;
 
 template <int MP, int STAGES>
 struct DecCfg {
   static constexpr int kSlot = MP * kBK;              // one k-block of the int8 activation
   static constexpr int kWindow = (96 * 1024) / kSlot; // k-blocks of activation kept resident
-  static constexpr size_t kSmem = static_cast<size_t>(STAGES) * kStageW + static_cast<size_t>(kWindow) * kSlot + 1024 + 256;
+  static constexpr int kStageOut = MP * kTileN * 2;  // bf16 output staging per epilogue set
+  static constexpr size_t kSmem = static_cast<size_t>(STAGES) * kStageW + static_cast<size_t>(kWindow) * kSlot +
+                                  2 * kStageOut + 1024 + 256;
   static constexpr int kTmemCols = 2 * MP < 32 ? 32 : 2 * MP;  // two accumulators
   static_assert(kSlot % 1024 == 0, "1 KiB alignment of activation slots");
   static_assert(kWindow >= STAGES, "the first window must cover the prefetched ring");
@@ -106,6 +108,46 @@ __device__ __forceinline__ void decode_epilogue_row(const int32_t (&acc)[MP], co
   }
 }
 
+// Epilogue of one 128-row tile for one set of four warps (all 128 threads call
+// it; `skip` suppresses a failed warp's work but not its barriers). bf16
+// outputs go through shared memory so that every token row leaves as 16-byte
+// stores; other outputs are written per element.
+template <int MP>
+__device__ __forceinline__ void decode_epilogue_tile(const int32_t (&acc)[MP], const float (&sx)[MP], int64_t M,
+                                                     int64_t N, int64_t tile, int row, int tid_set, int32_t z,
+                                                     const RowParams &rp, const EpilogueArgs &ep,
+                                                     uint16_t *stage, uint32_t bar_id, bool skip) {
+  const int64_t n = tile * kTileN + row;
+  if (ep.out_dtype != W8A8_BF16 || (N % 8) != 0) {
+    if (!skip) decode_epilogue_row<MP>(acc, sx, M, N, n, z, rp, ep);
+    return;
+  }
+  if (!skip && n < N) {
+#pragma unroll
+    for (int m = 0; m < MP; ++m) {
+      if (m < M) {
+        int32_t c = acc[m];
+        if (z != 0) c -= z * rp.cs;
+        const float y = __fmaf_rn(__int2float_rn(c), __fmul_rn(sx[m], rp.sw), rp.add);
+        const __nv_bfloat16 b = __float2bfloat16_rn(y);
+        stage[m * kTileN + row] = *reinterpret_cast<const uint16_t *>(&b);
+      }
+    }
+  }
+  __syncwarp();
+  named_barrier(bar_id, 128);
+  const int rows_out = static_cast<int>(M < MP ? M : MP);
+  uint16_t *out = static_cast<uint16_t *>(ep.out);
+  for (int c = tid_set; c < rows_out * (kTileN / 8); c += 128) {
+    const int m = c / (kTileN / 8), ch = c % (kTileN / 8);
+    const int64_t nn = tile * kTileN + ch * 8;
+    if (nn < N && !skip)
+      *reinterpret_cast<uint4 *>(out + m * N + nn) = *reinterpret_cast<const uint4 *>(stage + m * kTileN + ch * 8);
+  }
+  __syncwarp();
+  named_barrier(bar_id, 128);  // the staging buffer is reused by this set's next tile
+}
+
 // Position of a CTA in its run of units: the unit u = tile * nkb + kb, and
 // the index of kb in the activation window (k-blocks kb0, kb0+1, ... mod nkb).
 struct Cursor {
@@ -145,7 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sW = base;                            // STAGES x 16 KiB weight ring
   uint8_t *sX = sW + STAGES * kStageW;           // kWindow x MP*128 int8 activation, 128B swizzle
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sX + Cfg::kWindow * Cfg::kSlot);
+  uint16_t *sOut = reinterpret_cast<uint16_t *>(sX + Cfg::kWindow * Cfg::kSlot);  // 2 x MP x 128 bf16
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sOut) + 2 * Cfg::kStageOut);
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *xfull_bar = empty_bar + STAGES;      // activation window loaded
   uint64_t *xfree_bar = xfull_bar + 1;           // MMAs reading the window done
@@ -154,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *drain_bar = tempty_bar + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  volatile int *last_flag = abort_flag + 1;
+  volatile int *last_flag = abort_flag + 1;  // one per epilogue set
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -330,22 +373,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------ drain / epilogue
-    // The four warps meet at named barriers in the split-tile path, so after a
-    // failed wait a warp keeps walking the same segments (skipping the work)
-    // and still takes part in every barrier: no warp is ever left waiting.
+    // Two sets of four warps: set 0 drains accumulator 0 (even segments of the
+    // run), set 1 accumulator 1 (odd segments), so the flush of one segment
+    // overlaps the next. The four warps of a set meet at their own named
+    // barrier; after a failed wait a warp keeps walking the same segments
+    // (skipping the work) and still takes part in every barrier.
     pdl_wait_prerequisite();  // the previous kernel may still use the workspace or `out`
-    const int q = warp - kEpiWarp0;
+    const int set = (warp - kEpiWarp0) >> 2;
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    const int tid_set = threadIdx.x - (kEpiWarp0 + 4 * set) * 32;
+    const bool set_leader = tid_set == 0;
+    const uint32_t bar_id = 1 + set;
+    uint16_t *stage = sOut + set * (Cfg::kStageOut / 2);
     const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
     float sx[MP];
 #pragma unroll
     for (int m = 0; m < MP; ++m) sx[m] = (m < M) ? (ep.s_x_per_row ? __ldg(ep.S_x + m) : __ldg(ep.S_x)) : 0.0f;
-    int acc = 0;
+    const int acc = set;
     uint32_t acc_phase = 0;
     bool failed = false;
     int seg_idx = 0;
-    for (int64_t u = u_begin, tile = start.tile; u < u_end; ++tile) {
+    for (int64_t u = u_begin, tile = start.tile; u < u_end; ++tile, ++seg_idx) {
       const int64_t seg_end = u_end < (tile + 1) * nkb ? u_end : (tile + 1) * nkb;
       const int64_t seg_len = seg_end - u;
+      u = seg_end;
+      if ((seg_idx & 1) != set) continue;
       const int row = q * 32 + lane;  // weight row within the tile
       const int64_t n = tile * kTileN + row;
       const RowParams rp = load_row_params(n, N, z, ep);
@@ -359,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (threadIdx.x == kEpiWarp0 * 32 && seg_idx < 4) DTRACE(8 + 4 * seg_idx);
+      if (set_leader && seg_idx < 4) DTRACE(8 + 4 * seg_idx);
       int32_t v[MP];
 #pragma unroll
       for (int i = 0; i < MP; ++i) v[i] = 0;
@@ -383,13 +435,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty_bar[acc]);
       }
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
+      acc_phase ^= 1u;
 
       if (seg_len == nkb) {
-        if (!failed) decode_epilogue_row<MP>(v, sx, M, N, n, z, rp, ep);  // this CTA owns the whole tile
+        // this CTA owns the whole tile
+        decode_epilogue_tile<MP>(v, sx, M, N, tile, row, tid_set, z, rp, ep, stage, bar_id, failed);
       } else {
         // Split tile: add this run's partial sums to the tile's workspace slice
         // (red.global.add: exact and order-free); the CTA that brings the tile
@@ -402,49 +452,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (m < M) atomicAdd(p + m * kTileN + row, v[m]);
         }
         __syncwarp();
-        named_barrier(1, 128);
-        if (threadIdx.x == kEpiWarp0 * 32) {
+        named_barrier(bar_id, 128);
+        if (set_leader) {
           int last = 0;
           if (!*abort_flag) {
-            __threadfence();  // cumulative: orders the whole CTA's additions before the count
-            const uint32_t before = atomicAdd(counters + tile, static_cast<uint32_t>(seg_len));
+            // release: the CTA's additions (ordered before by the barrier) are
+            // visible before the count is
+            const uint32_t before = atomic_add_release_gpu(counters + tile, static_cast<uint32_t>(seg_len));
             last = (static_cast<int64_t>(before) + seg_len == nkb) ? 1 : 0;
-            if (last) __threadfence();
+            if (last) fence_acquire_gpu();  // ... and the last arriver sees every other CTA's
           }
-          *last_flag = last;
+          last_flag[set] = last;
           if (seg_idx < 4) {
             DTRACE(9 + 4 * seg_idx);
             DTRACE_VAL(10 + 4 * seg_idx, last);
           }
         }
         __syncwarp();
-        named_barrier(1, 128);
-        const bool last = *last_flag != 0;
-        if (last && !failed) {
+        named_barrier(bar_id, 128);
+        const bool last = last_flag[set] != 0;
+        if (last) {
+          if (!failed) {
 #pragma unroll
-          for (int m = 0; m < MP; ++m) {
-            if (m < M) {
-              v[m] = __ldcg(p + m * kTileN + row);
-              __stcg(p + m * kTileN + row, 0);  // leave the workspace zeroed for the next call
+            for (int m = 0; m < MP; ++m) {
+              if (m < M) {
+                v[m] = __ldcg(p + m * kTileN + row);
+                __stcg(p + m * kTileN + row, 0);  // leave the workspace zeroed for the next call
+              }
             }
           }
-          if (threadIdx.x == kEpiWarp0 * 32) {
+          if (set_leader) {
             int chk = 0;
 #pragma unroll
             for (int m = 0; m < MP; ++m) chk ^= v[m];
             DTRACE(24);  // the read-back has landed (chk depends on every load)
             DTRACE_VAL(25, chk);
           }
-          decode_epilogue_row<MP>(v, sx, M, N, n, z, rp, ep);
-          if (threadIdx.x == kEpiWarp0 * 32) DTRACE(26);
+          decode_epilogue_tile<MP>(v, sx, M, N, tile, row, tid_set, z, rp, ep, stage, bar_id, failed);
+          if (set_leader) {
+            DTRACE(26);
+            counters[tile] = 0u;  // zero again for the next call
+          }
         }
-        if (last && threadIdx.x == kEpiWarp0 * 32) counters[tile] = 0u;  // zero again for the next call
         __syncwarp();
-        named_barrier(1, 128);  // last_flag is rewritten by the next segment
+        named_barrier(bar_id, 128);  // last_flag is rewritten by this set's next segment
       }
-      if (threadIdx.x == kEpiWarp0 * 32 && seg_idx < 4) DTRACE(11 + 4 * seg_idx);
-      ++seg_idx;
-      u = seg_end;
+      if (set_leader && seg_idx < 4) DTRACE(11 + 4 * seg_idx);
     }
   }
 

@@ -621,9 +621,12 @@ cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_
                            const EpilogueArgs &ep, bool mixed, int num_sms, int32_t *status,
                            cudaStream_t s) {
   // CTA pairs (256-row tiles) once there are enough rows to fill them
+  // 7 stages of 32 KiB: the loaded L2/TMA latency is ~3000 cycles, and one
+  // stage is always being read by the MMAs, so six in flight keep the tensor
+  // pipe fed at 64 B/clk per SM.
   if (M >= 256 && num_sms >= 2) {
-    if (mixed) return launch_tc2_t<6, true>(Xq, Wq, M, N, K, ep, num_sms, status, s);
-    return launch_tc2_t<6, false>(Xq, Wq, M, N, K, ep, num_sms, status, s);
+    if (mixed) return launch_tc2_t<7, true>(Xq, Wq, M, N, K, ep, num_sms, status, s);
+    return launch_tc2_t<7, false>(Xq, Wq, M, N, K, ep, num_sms, status, s);
   }
   if (mixed) return launch_tc_t<256, 4, true>(Xq, Wq, M, N, K, ep, num_sms, status, s);
   return launch_tc_t<256, 4, false>(Xq, Wq, M, N, K, ep, num_sms, status, s);

@@ -32,9 +32,11 @@ struct EpilogueArgs {
 
 cudaError_t launch_quant_per_token(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                    int8_t *Xq, float *S_x, cudaStream_t s);
+// pdl = true: may start while the previous kernel runs; it waits for that
+// kernel before reading, then allows its own dependents to launch.
 cudaError_t launch_quant_per_tensor(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                     const float *r, const int32_t *Z, int8_t *Xq, int num_sms,
-                                    cudaStream_t s);
+                                    cudaStream_t s, bool pdl = false);
 cudaError_t launch_calibrate(const void *X, w8a8_dtype dt, int64_t T, int64_t K, int64_t ldx,
                              float *S, float *r, int32_t *Z, int num_sms, cudaStream_t s);
 cudaError_t launch_quant_weight(const void *W, w8a8_dtype dt, int64_t K, int64_t N, int64_t ldw,

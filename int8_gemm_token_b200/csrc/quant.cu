@@ -103,7 +103,12 @@ __global__ void __launch_bounds__(256) quant_per_tensor_kernel(const uint16_t *_
                                                                const float *__restrict__ r_ptr,
                                                                const int32_t *__restrict__ Z_ptr,
                                                                int8_t *__restrict__ Xq) {
-  pdl_launch_dependents();  // a decode GEMM launched after this one may start streaming weights
+  // When launched with programmatic stream serialization this kernel may start
+  // while the previous kernel still runs: wait for it before reading anything,
+  // and only then let the dependent decode GEMM start streaming its weights
+  // (everything before this kernel, weight writers included, is then complete).
+  pdl_wait_prerequisite();
+  pdl_launch_dependents();
   const float r = *r_ptr;
   const int z = *Z_ptr;
   const int64_t cpr = K >> 3;  // chunks per row
@@ -118,13 +123,21 @@ __global__ void __launch_bounds__(256) quant_per_tensor_kernel(const uint16_t *_
 
 cudaError_t launch_quant_per_tensor(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                     const float *r, const int32_t *Z, int8_t *Xq, int num_sms,
-                                    cudaStream_t s) {
+                                    cudaStream_t s, bool pdl) {
   const int64_t total = M * (K / 8);
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
-  quant_per_tensor_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(X, M, K, ldx, r, Z, Xq);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quant_per_tensor_kernel, X, M, K, ldx, r, Z, Xq);
 }
 
 // ------------------------------------------------------------ calibration
