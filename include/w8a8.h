@@ -147,15 +147,19 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
  *   colsum  device int32 [N]; required when Z != NULL
  *   s_w     device fp32 [N];  bias device fp32 [N] or NULL
  *   out     device [M, N] dense, out_dtype W8A8_BF16, W8A8_FP32 or W8A8_I32
- *   workspace/workspace_bytes: device scratch of at least
- *           w8a8_gemm_workspace_size(M, N, K) bytes (NULL allowed when it is 0).
- * M <= 32 (Decode-shaped) runs a split-K kernel that keeps per-tile counters
- * and int32 partial sums at the start of the workspace (the first
- * ceil(ceil(N/128) * 4 / 256) * 256 + ceil(N/128) * 16384 bytes). That region
- * must be zero before the first call that uses the workspace, and every call
- * that completes leaves it zero again, so one zero-filled workspace serves
- * every later call. Calls that overlap on the GPU must not share a workspace;
- * after a call that recorded a device error, zero the workspace again.
+ *   workspace/workspace_bytes: accepted for compatibility with
+ *           w8a8_linear_static and not used by this call (NULL/0 allowed).
+ * M <= 32 (Decode-shaped) runs a weight-streaming kernel: one cluster of up to
+ * 8 CTAs per 128 output channels splits K, and the partial int32 sums are
+ * added in distributed shared memory, so the call keeps no state in device
+ * memory between calls and calls on different streams may overlap.
+ * That kernel uses programmatic dependent launch: it may start while the
+ * previous kernel on the stream is still running, and it begins streaming Wq
+ * at once. Everything else (Xq, S_x, Z, colsum, s_w, bias, out) is touched
+ * only after the previous kernel has completed. So Wq, a constant weight,
+ * must not be written by a kernel that lets its dependents launch early
+ * (griddepcontrol.launch_dependents) and immediately precedes this call; no
+ * kernel of this library that writes Wq does so.
  */
 w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_per_row,
                               const int32_t *Z, const int8_t *Wq, const float *s_w,
@@ -163,12 +167,10 @@ w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
                               int64_t K, void *out, w8a8_dtype out_dtype, void *workspace,
                               size_t workspace_bytes, void *stream);
 
-/* Bytes of device workspace w8a8_gemm_dequant / w8a8_linear_static need for
- * this shape (enough for either call): for M <= 32 the tile counters
- * (ceil(N/128) * 4 bytes rounded up to 256), the split-K partial sums
- * (ceil(N/128) * 16 KiB), then M*K bytes (rounded up to 256) for the
- * statically quantized activation of w8a8_linear_static; for M > 32 only the
- * last part. */
+/* Bytes of device workspace w8a8_linear_static needs for this shape: M*K
+ * bytes rounded up to 256 for the statically quantized activation (no
+ * zero-fill needed; every byte read is written by the same call). Calls that
+ * overlap on the GPU must not share a workspace. */
 size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -177,7 +179,9 @@ size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * result as w8a8_quant_per_tensor followed by w8a8_gemm_dequant with
  * s_x_per_row = 0. For M <= 32 the GEMM kernel is launched with programmatic
  * dependent launch, so it streams the weight while the quantization kernel
- * runs and reads the quantized activation once that kernel has finished.
+ * (and the tail of the kernel before it) runs and reads the quantized
+ * activation once that kernel has finished; the rule on writing Wq given for
+ * w8a8_gemm_dequant applies.
  * Source: PDMIX glossary §2.2 (Decode has few tokens and is latency bound, so
  * a per-step quantization launch would be visible overhead) and §2.3 eq.
  * Q_decode; the hardware-acceleration chapter's note that decode is memory
@@ -201,13 +205,12 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
  * latency-critical step that cannot take an allocation's implicit device
  * synchronization. No counterpart on the pages: this is a deployment entry
  * point of this library.
- * The scratch (tile counters, partial sums, quantized activation) is one
- * fixed device array inside the library, 4,719,616 bytes, held by every GPU
- * that loads the library until the process exits. It serves M <= 32,
- * N <= 32768 and K <= 16384; larger shapes return W8A8_ERR_UNSUPPORTED_SHAPE
- * without launching anything. The call allocates nothing: it clears the part
- * of the array that must start at zero with cudaMemsetAsync on `stream`,
- * then launches the same kernels as w8a8_linear_static.
+ * The scratch (the quantized activation) is one fixed device array inside
+ * the library, 524,288 bytes (32 tokens x 16384), held by every GPU that
+ * loads the library until the process exits. It serves M <= 32, N <= 32768
+ * and K <= 16384; larger shapes return W8A8_ERR_UNSUPPORTED_SHAPE without
+ * launching anything. The call allocates nothing: it launches the same
+ * kernels as w8a8_linear_static with the array in place of the workspace.
  * The first call on a device also sets up that device (looks up the array's
  * device address and zero-fills it once, synchronously): make that first
  * call before any stream capture. All calls on a device share the one array,

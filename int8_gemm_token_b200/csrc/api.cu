@@ -205,9 +205,8 @@ static size_t align256(int64_t n) { return static_cast<size_t>(((n + 255) / 256)
 
 size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
-  // w8a8_linear_static keeps the statically quantized activation here (M*K bytes);
-  // the decode-shaped kernel (M <= 32) puts its tile counters and partial sums first.
-  if (M <= kDecodeMaxM) return decode_counters_bytes(N) + decode_partials_bytes(N) + align256(M * K);
+  // w8a8_linear_static keeps the statically quantized activation here; the
+  // GEMM kernels themselves need no workspace.
   return align256(M * K);
 }
 
@@ -234,11 +233,9 @@ w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
   if (w8a8_status s = check_gemm_common(Xq, Wq, s_w, bias, colsum, M, N, K, out, out_dtype)) return s;
   if (M == 0 || N == 0) return W8A8_OK;
   if (!S_x || (Z && !colsum)) return W8A8_ERR_INVALID_ARG;
+  (void)workspace;
+  (void)workspace_bytes;
   const bool decode = M <= kDecodeMaxM;
-  if (decode) {
-    if (!workspace || workspace_bytes < w8a8_gemm_workspace_size(M, N, K)) return W8A8_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return W8A8_ERR_MISALIGNED;
-  }
   DeviceInfo *d;
   if (w8a8_status s = device_info(&d)) return s;
   EpilogueArgs ep;
@@ -250,8 +247,8 @@ w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
   ep.bias = bias;
   ep.out = out;
   ep.out_dtype = out_dtype;
-  if (decode)  // ordinary stream order: the previous kernel may have written the weights
-    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, workspace, false, d->sm_count, d->status,
+  if (decode)
+    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, d->sm_count, d->status,
                                         static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_gemm_tc(Xq, Wq, M, N, K, ep, false, d->sm_count, d->status,
                                   static_cast<cudaStream_t>(stream)));
@@ -287,14 +284,15 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
   ep.out = out;
   ep.out_dtype = out_dtype;
   if (M <= kDecodeMaxM) {
-    // Static quantization into the workspace, then the decode GEMM launched with
-    // programmatic dependent launch: its weight stream starts while the
-    // quantization runs, and it reads the quantized activation after it.
-    int8_t *Xq = static_cast<int8_t *>(workspace) + decode_counters_bytes(N) + decode_partials_bytes(N);
+    // Static quantization into the workspace, then the decode GEMM; both use
+    // programmatic dependent launch, so the GEMM's weight stream starts while
+    // the quantization (and the previous kernel) run, and it reads the
+    // quantized activation once the quantization has completed.
+    int8_t *Xq = static_cast<int8_t *>(workspace);
     cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq, d->sm_count, st,
                                             /*pdl=*/true);
     if (e != cudaSuccess) return W8A8_ERR_CUDA;
-    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, workspace, true, d->sm_count, d->status, st));
+    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, d->sm_count, d->status, st));
   }
   int8_t *Xq = static_cast<int8_t *>(workspace);
   cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq,

@@ -32,8 +32,9 @@ struct EpilogueArgs {
 
 cudaError_t launch_quant_per_token(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                    int8_t *Xq, float *S_x, cudaStream_t s);
-// pdl = true: may start while the previous kernel runs; it waits for that
-// kernel before reading, then allows its own dependents to launch.
+// pdl = true: may start while the previous kernel runs. It lets its own
+// dependents (the decode GEMM) launch at once, then waits for the previous
+// kernel before reading or writing anything.
 cudaError_t launch_quant_per_tensor(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                     const float *r, const int32_t *Z, int8_t *Xq, int num_sms,
                                     cudaStream_t s, bool pdl = false);
@@ -50,19 +51,16 @@ cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_t s);
 
-// Decode-shaped GEMM (M <= 32): stream-K over the weight. The workspace holds
-// the per-tile counters (decode_counters_bytes(N)) and then the per-tile int32
-// partial sums (decode_partials_bytes(N)); both must be zero before the first
-// call and every completed call leaves them zero. pdl = true lets the kernel
-// start while the previous kernel in the stream runs: it streams weights at
-// once and waits for that kernel before reading Xq, the workspace or `out`
-// (so the previous kernel must not write Wq, s_w, colsum or bias).
+// Decode-shaped GEMM (M <= 32): one cluster of decode_split(N, K, num_sms)
+// CTAs per 128-row weight tile, partial sums reduced through distributed
+// shared memory (no workspace). Launched with programmatic dependent launch:
+// it may start while the previous kernel in the stream runs, streams its first
+// weight tiles at once and waits for that kernel before reading Xq or S_x,
+// s_w, colsum, bias and before writing `out` (so a kernel that lets its
+// dependents launch early must not write Wq).
 cudaError_t launch_gemm_decode(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
-                               const EpilogueArgs &ep, void *workspace, bool pdl, int num_sms, int32_t *status,
-                               cudaStream_t s);
-size_t decode_counters_bytes(int64_t N);
-size_t decode_partials_bytes(int64_t N);
-int decode_grid(int64_t N, int64_t K, int num_sms);
+                               const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s);
+int decode_split(int64_t N, int64_t K, int num_sms);
 
 // LLM.int8() outlier split: column-flag pass into a K-bit bitmap in
 // `workspace` (outlier_workspace_bytes(K); zeroed by the launcher), then the

@@ -6,10 +6,10 @@
 // is not a stream operation and breaks the capture), a plug-in running inside
 // another runtime that owns all device memory, or a latency-critical step
 // where an allocation's implicit device synchronization is not acceptable.
-// This entry point needs no memory from them: its scratch (split-K tile
-// counters and partial sums, and the statically quantized activation) lives
-// in one file-scope device array of fixed size, which every GPU that loads
-// the library holds until the process exits.
+// This entry point needs no memory from them: its scratch (the statically
+// quantized activation handed from the quantization kernel to the GEMM)
+// lives in one file-scope device array of fixed size, which every GPU that
+// loads the library holds until the process exits.
 #include <mutex>
 
 #include "device.cuh"
@@ -23,9 +23,8 @@ namespace {
 constexpr int64_t kNoAllocMaxM = 32;
 constexpr int64_t kNoAllocMaxN = 32768;
 constexpr int64_t kNoAllocMaxK = 16384;
-// counters (256 tiles x 4 B, rounded to 256 B) + partial sums (256 tiles x 16 KiB)
-// + quantized activation (32 x 16384 B) = 4,719,616 bytes.
-constexpr size_t kNoAllocScratchBytes = 1024 + 256 * 16384 + 32 * 16384;
+// the quantized activation, 32 tokens x 16384 bytes = 524,288 bytes.
+constexpr size_t kNoAllocScratchBytes = kNoAllocMaxM * kNoAllocMaxK;
 
 // One array per device (each device that loads the library holds its own
 // copy). In host code this name is only a stand-in for the symbol, never a
@@ -37,8 +36,7 @@ std::mutex g_setup_mutex;
 void *g_scratch_ptr[kMaxDevices] = {};
 
 // Once per device, with that device current: the device address of the
-// scratch array, and one zero fill (the tile counters and partial sums must
-// start at zero).
+// scratch array (zero-filled once, so it never holds stale bytes).
 w8a8_status scratch_for_current_device(void **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -90,12 +88,9 @@ extern "C" w8a8_status w8a8_linear_static_noalloc(const void *X, int64_t M, int6
   if (w8a8_status s = scratch_for_current_device(&scratch)) return s;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t zero_bytes = decode_counters_bytes(N) + decode_partials_bytes(N);
-  // Completed calls leave counters and partial sums at zero; clearing them on
-  // the stream as well keeps a call correct after one that failed part-way.
-  if (cudaMemsetAsync(scratch, 0, zero_bytes, st) != cudaSuccess) return W8A8_ERR_CUDA;
-  int8_t *Xq = static_cast<int8_t *>(scratch) + zero_bytes;
-  if (launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq, sms, st) != cudaSuccess)
+  int8_t *Xq = static_cast<int8_t *>(scratch);  // every byte read is written first by this call
+  if (launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq, sms, st, /*pdl=*/true) !=
+      cudaSuccess)
     return W8A8_ERR_CUDA;
   EpilogueArgs ep;
   ep.S_x = S;
@@ -106,6 +101,5 @@ extern "C" w8a8_status w8a8_linear_static_noalloc(const void *X, int64_t M, int6
   ep.bias = bias;
   ep.out = out;
   ep.out_dtype = out_dtype;
-  return launch_gemm_decode(Xq, K, Wq, M, N, K, ep, scratch, true, sms, status, st) == cudaSuccess ? W8A8_OK
-                                                                                                 : W8A8_ERR_CUDA;
+  return launch_gemm_decode(Xq, K, Wq, M, N, K, ep, sms, status, st) == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA;
 }

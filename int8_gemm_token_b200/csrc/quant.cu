@@ -104,11 +104,12 @@ __global__ void __launch_bounds__(256) quant_per_tensor_kernel(const uint16_t *_
                                                                const int32_t *__restrict__ Z_ptr,
                                                                int8_t *__restrict__ Xq) {
   // When launched with programmatic stream serialization this kernel may start
-  // while the previous kernel still runs: wait for it before reading anything,
-  // and only then let the dependent decode GEMM start streaming its weights
-  // (everything before this kernel, weight writers included, is then complete).
-  pdl_wait_prerequisite();
+  // while the previous kernel still runs. It lets the dependent decode GEMM
+  // launch at once (that GEMM streams only the weight before its own wait,
+  // which returns after this kernel has completed), then waits for the
+  // previous kernel before reading X or writing Xq.
   pdl_launch_dependents();
+  pdl_wait_prerequisite();
   const float r = *r_ptr;
   const int z = *Z_ptr;
   const int64_t cpr = K >> 3;  // chunks per row

@@ -160,20 +160,19 @@ def w8a8_gemm_workspace_size(M: int, N: int, K: int) -> int:
 
 
 def new_workspace(M: int, N: int, K: int, device=None) -> torch.Tensor | None:
-    """A zero-filled workspace for w8a8_gemm_dequant / w8a8_linear_static of
-    this shape (None when the shape needs none). Calls that complete leave it
-    zero-filled, so one workspace serves every later call on the same stream."""
+    """A workspace for w8a8_linear_static of this shape (None when the shape
+    needs none). It needs no initial contents; calls on one stream may share it."""
     n = w8a8_gemm_workspace_size(M, N, K)
     if n == 0:
         return None
-    return torch.zeros((n,), dtype=torch.uint8, device=device or torch.device("cuda"))
+    return torch.empty((n,), dtype=torch.uint8, device=device or torch.device("cuda"))
 
 
 def _workspace(n: int, dev, ws):
     if n == 0:
         return None, 0
     if ws is None:
-        ws = torch.zeros((n,), dtype=torch.uint8, device=dev)
+        ws = torch.empty((n,), dtype=torch.uint8, device=dev)
     return ws, ws.numel() * ws.element_size()
 
 
@@ -188,8 +187,7 @@ def w8a8_gemm_dequant(Xq, S_x, Wq, s_w, colsum=None, Z=None, bias=None, out=None
     if S_x.numel() not in (1, M):
         raise ValueError("S_x holds one scale per row or a single per-tensor scale")
     per_row = 1 if S_x.numel() == M else 0
-    # only the decode-shaped kernel (M <= 32) uses a workspace in this call
-    ws, nbytes = _workspace(w8a8_gemm_workspace_size(M, N, K) if M <= DECODE_MAX_M else 0, Xq.device, workspace)
+    ws, nbytes = (None, 0) if workspace is None else (workspace, workspace.numel() * workspace.element_size())
     _check("w8a8_gemm_dequant", lib().w8a8_gemm_dequant(
         _ptr(Xq), _ptr(S_x), per_row, _ptr(Z), _ptr(Wq), _ptr(s_w), _ptr(colsum), _ptr(bias),
         M, N, K, _ptr(out), _dt(out.dtype), _ptr(ws), nbytes, _stream(stream)))
