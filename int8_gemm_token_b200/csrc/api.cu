@@ -248,7 +248,7 @@ w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
   ep.out = out;
   ep.out_dtype = out_dtype;
   if (decode)
-    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, d->sm_count, d->status,
+    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, d->status,
                                         static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_gemm_tc(Xq, Wq, M, N, K, ep, false, d->sm_count, d->status,
                                   static_cast<cudaStream_t>(stream)));
@@ -292,7 +292,7 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
     cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq, d->sm_count, st,
                                             /*pdl=*/true);
     if (e != cudaSuccess) return W8A8_ERR_CUDA;
-    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, d->sm_count, d->status, st));
+    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, d->status, st));
   }
   int8_t *Xq = static_cast<int8_t *>(workspace);
   cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq,

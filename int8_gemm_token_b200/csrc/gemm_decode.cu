@@ -35,6 +35,8 @@
 //     quantization kernel and the tail of the previous decode GEMM. The
 //     weight is the one operand read before that wait; the activation, the
 //     scales and the output are touched only after it.
+#include <atomic>
+
 #include "device.cuh"
 #include "kernels.h"
 
@@ -50,16 +52,145 @@ constexpr int kEpiWarp0 = 4;
 constexpr int kCtasPerSm = 2;            // two CTAs of ~100 KiB share an SM
 constexpr int kMaxSplit = 8;
 
-template <int MP>
+// First weight row of a tile that cluster rank j finishes (j = SPLIT gives the
+// end of the tile): j * 128 / SPLIT rounded down to a multiple of 8, so that
+// every owner's rows start on a 16-byte boundary of the output.
+template <int SPLIT>
+__host__ __device__ constexpr int owner_row0(int j) {
+  return j >= SPLIT ? kTileN : ((j * kTileN / SPLIT) & ~7);
+}
+
+template <int SPLIT>
+constexpr int max_owned_rows() {
+  int r = 0;
+  for (int j = 0; j < SPLIT; ++j) {
+    const int d = owner_row0<SPLIT>(j + 1) - owner_row0<SPLIT>(j);
+    if (d > r) r = d;
+  }
+  return r;
+}
+
+template <int MP, int SPLIT>
 struct DecCfg {
   static constexpr int kStageX = MP * kBK;  // int8 activation k-block
-  // ring depth: as deep as two CTAs per SM allow (228 KiB per SM, 1 KiB reserved per CTA)
-  static constexpr int kStages = MP == 16 ? 6 : 5;
-  static constexpr size_t kSmem = static_cast<size_t>(kStages) * (kStageW + kStageX) + 1024 + 256;
+  static constexpr int kStage = kStageW + kStageX;
+  // weight rows one CTA finishes, at most (a multiple of 8)
+  static constexpr int kR = max_owned_rows<SPLIT>();
+  // partial sums this CTA receives from the other SPLIT-1 CTAs of its cluster
+  static constexpr int kRedBytes = (SPLIT - 1) * MP * kR * 4;
+  // two CTAs per SM: 228 KiB per SM, 1 KiB of it reserved per CTA
+  static constexpr int kBudget = 228 * 1024 / kCtasPerSm - 1024 - 1024 /*alignment slack*/ - 256 /*barriers*/;
+  static constexpr int kStagesFit = (kBudget - kRedBytes) / kStage;
+  static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
+  static constexpr size_t kSmem = static_cast<size_t>(kStages) * kStage + kRedBytes + 1024 + 256;
   static constexpr int kTmemCols = 32;
+  static_assert(kR % 8 == 0, "owned rows in 8-row groups");
   static_assert(kStageX % 1024 == 0, "1 KiB alignment of activation stages");
+  static_assert(kStages >= 3, "ring depth");
+  static_assert(MP * kR * 4 <= kStages * kStageW, "this CTA's own partial sums fit in the weight ring");
   static_assert(kCtasPerSm * (kSmem + 1024) <= 228 * 1024, "two CTAs per SM");
 };
+
+// 8 consecutive int32 from this CTA's shared memory (32-byte aligned address).
+__device__ __forceinline__ void ld_shared_8(uint32_t addr, int32_t (&v)[8]) {
+  asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+               : "r"(addr));
+  asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(addr + 16));
+}
+
+// Per-channel constants of outputs n0 .. n0+7 (n0 a multiple of 8; zero past N).
+struct Consts8 {
+  float sw[8], bs[8];
+  int32_t cs[8];
+};
+
+__device__ __forceinline__ void load_consts8(const EpilogueArgs &ep, int64_t n0, int64_t N, int32_t z, Consts8 &k) {
+  if (n0 + 8 <= N) {
+    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(ep.s_w + n0));
+    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(ep.s_w + n0) + 1);
+    k.sw[0] = w0.x; k.sw[1] = w0.y; k.sw[2] = w0.z; k.sw[3] = w0.w;
+    k.sw[4] = w1.x; k.sw[5] = w1.y; k.sw[6] = w1.z; k.sw[7] = w1.w;
+    if (ep.bias) {
+      const float4 b0 = __ldg(reinterpret_cast<const float4 *>(ep.bias + n0));
+      const float4 b1 = __ldg(reinterpret_cast<const float4 *>(ep.bias + n0) + 1);
+      k.bs[0] = b0.x; k.bs[1] = b0.y; k.bs[2] = b0.z; k.bs[3] = b0.w;
+      k.bs[4] = b1.x; k.bs[5] = b1.y; k.bs[6] = b1.z; k.bs[7] = b1.w;
+    }
+    if (z != 0) {
+      const int4 c0 = __ldg(reinterpret_cast<const int4 *>(ep.colsum + n0));
+      const int4 c1 = __ldg(reinterpret_cast<const int4 *>(ep.colsum + n0) + 1);
+      k.cs[0] = c0.x; k.cs[1] = c0.y; k.cs[2] = c0.z; k.cs[3] = c0.w;
+      k.cs[4] = c1.x; k.cs[5] = c1.y; k.cs[6] = c1.z; k.cs[7] = c1.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool ok = n0 + i < N;
+      k.sw[i] = ok ? __ldg(ep.s_w + n0 + i) : 0.0f;
+      k.bs[i] = (ok && ep.bias) ? __ldg(ep.bias + n0 + i) : 0.0f;
+      k.cs[i] = (ok && z != 0) ? __ldg(ep.colsum + n0 + i) : 0;
+    }
+  }
+}
+
+// The epilogue of 8 consecutive outputs out[m, n0 .. n0+7] (n0 a multiple of
+// 8), each in the fixed order of include/w8a8.h:
+// c = acc - Z*colsum[n]; y = fmaf(float(c), S_x[m]*s_w[n], bias[n]).
+__device__ __forceinline__ void epilogue8(const EpilogueArgs &ep, int64_t m, int64_t n0, int64_t N,
+                                          const int32_t (&a)[8], int32_t z, float sx, const Consts8 &k) {
+  const bool full = n0 + 8 <= N;
+  int32_t c[8];
+  float y[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = z != 0 ? a[i] - z * k.cs[i] : a[i];
+    float add = 0.0f;
+    if (ep.bias) add = __fadd_rn(add, k.bs[i]);
+    y[i] = __fmaf_rn(__int2float_rn(c[i]), __fmul_rn(sx, k.sw[i]), add);
+  }
+  const int64_t o = m * N + n0;
+  if (ep.out_dtype == W8A8_BF16) {
+    uint16_t *out = static_cast<uint16_t *>(ep.out) + o;
+    if (full && (o % 8) == 0) {
+      uint4 v;
+      v.x = pack_bf16x2(y[0], y[1]);
+      v.y = pack_bf16x2(y[2], y[3]);
+      v.z = pack_bf16x2(y[4], y[5]);
+      v.w = pack_bf16x2(y[6], y[7]);
+      *reinterpret_cast<uint4 *>(out) = v;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (n0 + i < N) {
+          __nv_bfloat16 b = __float2bfloat16_rn(y[i]);
+          out[i] = *reinterpret_cast<uint16_t *>(&b);
+        }
+    }
+  } else if (ep.out_dtype == W8A8_FP32) {
+    float *out = static_cast<float *>(ep.out) + o;
+    if (full && (o % 4) == 0) {
+      reinterpret_cast<float4 *>(out)[0] = make_float4(y[0], y[1], y[2], y[3]);
+      reinterpret_cast<float4 *>(out)[1] = make_float4(y[4], y[5], y[6], y[7]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (n0 + i < N) out[i] = y[i];
+    }
+  } else {
+    int32_t *out = static_cast<int32_t *>(ep.out) + o;
+    if (full && (o % 4) == 0) {
+      reinterpret_cast<int4 *>(out)[0] = make_int4(c[0], c[1], c[2], c[3]);
+      reinterpret_cast<int4 *>(out)[1] = make_int4(c[4], c[5], c[6], c[7]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (n0 + i < N) out[i] = c[i];
+    }
+  }
+}
 
 // Store a 32-bit word to a shared::cluster address (from map_to_rank).
 __device__ __forceinline__ void st_shared_cluster(uint32_t addr, uint32_t v) {
@@ -71,13 +202,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     gemm_i8_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                           int64_t M, int64_t N, int64_t K, const __grid_constant__ EpilogueArgs ep,
                           int32_t *status, uint64_t limit_ns) {
-  using Cfg = DecCfg<MP>;
+  using Cfg = DecCfg<MP, SPLIT>;
   constexpr uint32_t kIdesc = idesc_i8(kTileN, MP);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sW = base;                            // kStages x 16 KiB weight ring
   uint8_t *sX = sW + Cfg::kStages * kStageW;     // kStages x MP*128 activation ring
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sX + Cfg::kStages * Cfg::kStageX);
+  int32_t *sRed = reinterpret_cast<int32_t *>(sX + Cfg::kStages * Cfg::kStageX);  // [SPLIT-1][MP][kR]
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sX + Cfg::kStages * Cfg::kStageX + Cfg::kRedBytes);
   uint64_t *empty_bar = full_bar + Cfg::kStages;
   uint64_t *tfull_bar = empty_bar + Cfg::kStages;
   uint64_t *drain_bar = tfull_bar + 1;
@@ -193,34 +325,23 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   }
 
-  // ------------------------------------------------ epilogue warps
-  // This CTA finishes rows [r0, r0 + nrows) of the tile: epilogue thread t
-  // takes row r0 + t % nrows for tokens t / nrows, + groups, + 2 groups, ...
-  const int r0 = static_cast<int>(rank) * kTileN / SPLIT;
-  const int nrows = (static_cast<int>(rank) + 1) * kTileN / SPLIT - r0;
-  const int groups = kTileN / nrows;
+  // ------------------------------------------------ partial sums -> shared memory
+  // Epilogue thread t holds row t of the tile (its TMEM lane). Rows
+  // [owner_row0(j), owner_row0(j+1)) are finished by cluster rank j: the
+  // owner keeps its own partial sums in its (now idle) weight ring, the other
+  // ranks store theirs into the owner's sRed.
   const int t = threadIdx.x - kEpiWarp0 * 32;  // epilogue thread index (negative elsewhere)
-  const int g = t / nrows;
-  const int rl = r0 + t % nrows;
-  const int64_t n = tile * kTileN + rl;
+  uint32_t owner = 0;
+#pragma unroll
+  for (int j = 1; j < SPLIT; ++j)
+    if (t >= owner_row0<SPLIT>(j)) owner = static_cast<uint32_t>(j);
+  const int owner_r0 = owner_row0<SPLIT>(static_cast<int>(owner));
   const int rows_m = static_cast<int>(M < MP ? M : MP);
-  const bool finisher = t >= 0 && g < groups && n < N;
-  uint32_t acc[MP];
-  int32_t zc = 0;
-  float sw = 0.0f, add = 0.0f, sx0 = 0.0f;
-  bool ready = true;
+  int32_t *sOwn = reinterpret_cast<int32_t *>(sW);  // [MP][kR], once this CTA's MMAs are done
   if (warp >= kEpiWarp0) {
-    pdl_wait_prerequisite();  // the previous kernel may still read `out` or write S_x, s_w, ...
-    // per-channel constants, fetched while the weight still streams
-    if (finisher) {
-      const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
-      if (z != 0) zc = z * __ldg(ep.colsum + n);
-      sw = __ldg(ep.s_w + n);
-      if (ep.bias) add = __fadd_rn(add, __ldg(ep.bias + n));
-      sx0 = __ldg(ep.S_x);
-    }
-    // tfull also means every MMA has finished reading the weight ring
-    ready = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(tfull_bar, 0, abort_flag, limit_ns));
+    pdl_wait_prerequisite();  // the bounded wait below counts from here, not from an early launch
+    // tfull: every MMA of this CTA has completed (the weight ring is idle)
+    const bool ready = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(tfull_bar, 0, abort_flag, limit_ns));
     if (!ready) {
       if (lane == 0) {
         record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
@@ -228,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
     } else {
       tc_fence_after();
+      uint32_t acc[MP];
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>((warp - kEpiWarp0) * 32) << 16);
       if constexpr (MP == 32)
         tmem_ld_32x32b_x32(taddr, acc);
@@ -235,57 +357,62 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         tmem_ld_32x32b_x16(taddr, acc);
       tmem_ld_wait();
       tc_fence_before();
+      if (owner == rank) {
+#pragma unroll
+        for (int m = 0; m < MP; ++m)
+          if (m < rows_m) sOwn[m * Cfg::kR + (t - owner_r0)] = static_cast<int32_t>(acc[m]);
+      } else {
+        // sRed[slot][m][row - owner_row0(owner)] of the owner
+        const int slot = static_cast<int>(rank < owner ? rank : rank - 1);
+        const uint32_t dst = map_to_rank(sRed + slot * MP * Cfg::kR + (t - owner_r0), owner);
+#pragma unroll
+        for (int m = 0; m < MP; ++m)
+          if (m < rows_m) st_shared_cluster(dst + 4u * static_cast<uint32_t>(m * Cfg::kR), acc[m]);
+      }
     }
   }
+  // Thread i finishes chunks of 8 outputs (token m, 8 consecutive owned rows);
+  // the constants of its first chunk are fetched before the barrier.
+  pdl_wait_prerequisite();  // the previous kernel may still read `out` or write S_x, s_w, ...
+  const int r0 = owner_row0<SPLIT>(static_cast<int>(rank));
+  const int per_m = (owner_row0<SPLIT>(static_cast<int>(rank) + 1) - r0) / 8;
+  const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
+  const float sx0 = ep.s_x_per_row ? 0.0f : __ldg(ep.S_x);
+  Consts8 k0;
+  {
+    const int m = static_cast<int>(threadIdx.x) / per_m;
+    const int64_t n0 = tile * kTileN + r0 + 8 * (static_cast<int>(threadIdx.x) - m * per_m);
+    if (static_cast<int>(threadIdx.x) < rows_m * per_m && n0 < N) load_consts8(ep, n0, N, z, k0);
+  }
+  __syncwarp();
+  if constexpr (SPLIT > 1)
+    cluster_sync_all();  // every partial sum has landed (release / acquire); no remote access after this
+  else
+    __syncthreads();
 
-  // One output element in the fixed order of include/w8a8.h:
-  // c = acc - Z*colsum[n]; y = fmaf(float(c), S_x[m]*s_w[n], bias[n]).
-  auto store = [&](int m, int32_t a) {
-    const int32_t c = a - zc;
-    const float sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : sx0;
-    const float y = __fmaf_rn(__int2float_rn(c), __fmul_rn(sx, sw), add);
-    const int64_t o = static_cast<int64_t>(m) * N + n;
-    if (ep.out_dtype == W8A8_BF16)
-      static_cast<__nv_bfloat16 *>(ep.out)[o] = __float2bfloat16_rn(y);
-    else if (ep.out_dtype == W8A8_FP32)
-      static_cast<float *>(ep.out)[o] = y;
-    else
-      static_cast<int32_t *>(ep.out)[o] = c;
-  };
-
-  if constexpr (SPLIT == 1) {
-    // thread t holds row t (its TMEM lane) for every token: store directly
-    if (finisher && ready && !*abort_flag) {
+  // ------------------------------------------------ sum + epilogue, all threads
+  if (!*abort_flag) {
+    for (int idx = threadIdx.x; idx < rows_m * per_m; idx += kThreads) {
+      const int m = idx / per_m;
+      const int rl = 8 * (idx - m * per_m);  // first of the 8 rows, within this CTA's rows
+      const int64_t n0 = tile * kTileN + r0 + rl;
+      if (n0 >= N) continue;
+      Consts8 kc;
+      if (idx == static_cast<int>(threadIdx.x))
+        kc = k0;
+      else
+        load_consts8(ep, n0, N, z, kc);
+      int32_t a[8];
+      ld_shared_8(smem_addr(sOwn + m * Cfg::kR + rl), a);
+#pragma unroll 2
+      for (int j = 0; j < SPLIT - 1; ++j) {
+        int32_t p[8];
+        ld_shared_8(smem_addr(sRed + (j * MP + m) * Cfg::kR + rl), p);
 #pragma unroll
-      for (int m = 0; m < MP; ++m)
-        if (m < rows_m) store(m, static_cast<int32_t>(acc[m]));
-    }
-  } else {
-    // Partial sums of the cluster, gathered in the owner's shared memory:
-    // sRed[s][m][row - r0 of the owner] holds CTA s's sum for token m.
-    constexpr int kR = (kTileN + SPLIT - 1) / SPLIT;
-    static_assert(SPLIT * MP * kR * 4 <= Cfg::kStages * kStageW, "the partial sums reuse the weight ring");
-    int32_t *sRed = reinterpret_cast<int32_t *>(sW);
-    __syncwarp();
-    cluster_sync_all();  // every MMA of the cluster is done: the weight rings are free
-    if (warp >= kEpiWarp0 && ready) {
-      const int row = t;  // this thread's TMEM lane
-      const uint32_t owner = static_cast<uint32_t>(((row + 1) * SPLIT - 1) / kTileN);
-      const int owner_r0 = static_cast<int>(owner) * kTileN / SPLIT;
-      const uint32_t dst = map_to_rank(sRed + (static_cast<int>(rank) * MP) * kR + (row - owner_r0), owner);
-#pragma unroll
-      for (int m = 0; m < MP; ++m)
-        if (m < rows_m) st_shared_cluster(dst + 4u * static_cast<uint32_t>(m * kR), acc[m]);
-    }
-    __syncwarp();
-    cluster_sync_all();  // every partial sum has landed (release / acquire)
-    if (finisher && !*abort_flag) {
-      for (int m = g; m < rows_m; m += groups) {
-        int32_t a = 0;
-#pragma unroll
-        for (int j = 0; j < SPLIT; ++j) a += sRed[(j * MP + m) * kR + (rl - r0)];
-        store(m, a);
+        for (int i = 0; i < 8; ++i) a[i] += p[i];
       }
+      const float sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : sx0;
+      epilogue8(ep, m, n0, N, a, z, sx, kc);
     }
   }
 
@@ -298,10 +425,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
 }
 
+// Dynamic shared memory of the kernel, and the largest shared-memory carveout:
+// without it the driver may size the carveout for one CTA per SM.
+template <int MP, int SPLIT>
+cudaError_t configure_decode_kernel() {
+  auto kern = gemm_i8_decode_kernel<MP, SPLIT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(DecCfg<MP, SPLIT>::kSmem));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
+
 template <int MP, int SPLIT>
 cudaError_t launch_decode_t(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                             const EpilogueArgs &ep, int32_t *status, cudaStream_t s) {
-  using Cfg = DecCfg<MP>;
+  using Cfg = DecCfg<MP, SPLIT>;
   alignas(64) CUtensorMap tmW, tmX;
   if (!encode_tmap_2d(&tmW, Wq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                       static_cast<uint64_t>(K), kBK, kTileN, true))
@@ -310,8 +448,7 @@ cudaError_t launch_decode_t(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int
                       static_cast<uint64_t>(ldx), kBK, MP, true))
     return cudaErrorInvalidValue;
   auto kern = gemm_i8_decode_kernel<MP, SPLIT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(Cfg::kSmem));
+  cudaError_t e = configure_decode_kernel<MP, SPLIT>();
   if (e != cudaSuccess) return e;
   const int64_t tiles = (N + kTileN - 1) / kTileN;
   cudaLaunchConfig_t cfg = {};
@@ -331,10 +468,82 @@ cudaError_t launch_decode_t(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int
   return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, M, N, K, ep, status, kWaitLimitNs);
 }
 
+// A kernel with the decode kernel's launch shape and no body. The runtime's
+// occupancy answer for the decode kernel itself is one CTA per SM (it
+// allocates tensor memory), while the hardware runs two of its CTAs per SM
+// (32 TMEM columns each); the answer for this stand-in gives how clusters of a
+// CTA of that size pack into the GPCs.
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_occupancy_standin() {}
+
+// Clusters of SPLIT decode CTAs that can be resident at once on the current
+// device (cached per device).
+template <int MP, int SPLIT>
+int max_active_clusters() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return 0;
+  }
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  using Cfg = DecCfg<MP, SPLIT>;
+  if (cudaFuncSetAttribute(decode_occupancy_standin, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           200 * 1024) != cudaSuccess ||
+      cudaFuncSetAttribute(decode_occupancy_standin, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(SPLIT);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = SPLIT;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_occupancy_standin, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+template <int MP>
+int max_active_clusters_of(int split) {
+  switch (split) {
+    case 8: return max_active_clusters<MP, 8>();
+    case 7: return max_active_clusters<MP, 7>();
+    case 6: return max_active_clusters<MP, 6>();
+    case 5: return max_active_clusters<MP, 5>();
+    case 4: return max_active_clusters<MP, 4>();
+    case 3: return max_active_clusters<MP, 3>();
+    case 2: return max_active_clusters<MP, 2>();
+    default: return max_active_clusters<MP, 1>();
+  }
+}
+
+// Largest cluster size (1..8) whose clusters, one per 128-row tile, are all
+// resident at once, with at least 2 k-blocks per CTA.
+template <int MP>
+int decode_split_mp(int64_t N, int64_t K) {
+  const int64_t tiles = (N + kTileN - 1) / kTileN;
+  const int64_t nkb = (K + kBK - 1) / kBK;
+  for (int s = kMaxSplit; s >= 2; --s)
+    if (nkb >= 2 * s && tiles <= max_active_clusters_of<MP>(s)) return s;
+  return 1;
+}
+
 template <int MP>
 cudaError_t launch_decode_mp(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
-                             const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
-  switch (decode_split(N, K, num_sms)) {
+                             const EpilogueArgs &ep, int32_t *status, cudaStream_t s) {
+  switch (decode_split_mp<MP>(N, K)) {
     case 8: return launch_decode_t<MP, 8>(Xq, ldx, Wq, M, N, K, ep, status, s);
     case 7: return launch_decode_t<MP, 7>(Xq, ldx, Wq, M, N, K, ep, status, s);
     case 6: return launch_decode_t<MP, 6>(Xq, ldx, Wq, M, N, K, ep, status, s);
@@ -348,21 +557,14 @@ cudaError_t launch_decode_mp(const int8_t *Xq, int64_t ldx, const int8_t *Wq, in
 
 }  // namespace
 
-// Largest cluster size (1..8) with tiles * size within one wave of CTAs (two
-// per SM) and at least 2 k-blocks per CTA.
-int decode_split(int64_t N, int64_t K, int num_sms) {
-  const int64_t tiles = (N + kTileN - 1) / kTileN;
-  const int64_t nkb = (K + kBK - 1) / kBK;
-  int split = 1;
-  for (int s = 2; s <= kMaxSplit; ++s)
-    if (tiles * s <= static_cast<int64_t>(kCtasPerSm) * num_sms && nkb >= 2 * s) split = s;
-  return split;
+int decode_split(int64_t M, int64_t N, int64_t K) {
+  return M <= 16 ? decode_split_mp<16>(N, K) : decode_split_mp<32>(N, K);
 }
 
 cudaError_t launch_gemm_decode(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
-                               const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
-  if (M <= 16) return launch_decode_mp<16>(Xq, ldx, Wq, M, N, K, ep, num_sms, status, s);
-  return launch_decode_mp<32>(Xq, ldx, Wq, M, N, K, ep, num_sms, status, s);
+                               const EpilogueArgs &ep, int32_t *status, cudaStream_t s) {
+  if (M <= 16) return launch_decode_mp<16>(Xq, ldx, Wq, M, N, K, ep, status, s);
+  return launch_decode_mp<32>(Xq, ldx, Wq, M, N, K, ep, status, s);
 }
 
 }  // namespace w8a8

@@ -51,16 +51,17 @@ cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_t s);
 
-// Decode-shaped GEMM (M <= 32): one cluster of decode_split(N, K, num_sms)
-// CTAs per 128-row weight tile, partial sums reduced through distributed
-// shared memory (no workspace). Launched with programmatic dependent launch:
-// it may start while the previous kernel in the stream runs, streams its first
+// Decode-shaped GEMM (M <= 32): one cluster of decode_split(M, N, K) CTAs
+// per 128-row weight tile, partial sums reduced through distributed shared
+// memory (no workspace). Launched with programmatic dependent launch: it may
+// start while the previous kernel in the stream runs, streams its first
 // weight tiles at once and waits for that kernel before reading Xq or S_x,
 // s_w, colsum, bias and before writing `out` (so a kernel that lets its
 // dependents launch early must not write Wq).
 cudaError_t launch_gemm_decode(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
-                               const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s);
-int decode_split(int64_t N, int64_t K, int num_sms);
+                               const EpilogueArgs &ep, int32_t *status, cudaStream_t s);
+// Cluster size the decode GEMM uses for this shape on the current device.
+int decode_split(int64_t M, int64_t N, int64_t K);
 
 // LLM.int8() outlier split: column-flag pass into a K-bit bitmap in
 // `workspace` (outlier_workspace_bytes(K); zeroed by the launcher), then the

@@ -101,5 +101,5 @@ extern "C" w8a8_status w8a8_linear_static_noalloc(const void *X, int64_t M, int6
   ep.bias = bias;
   ep.out = out;
   ep.out_dtype = out_dtype;
-  return launch_gemm_decode(Xq, K, Wq, M, N, K, ep, sms, status, st) == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA;
+  return launch_gemm_decode(Xq, K, Wq, M, N, K, ep, status, st) == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA;
 }

@@ -73,7 +73,8 @@ def test_outlier_split_thresholds_and_overflow():
 
 @pytest.mark.parametrize("M,K,N,cols", [(16, 256, 512, [3, 200]), (300, 400, 520, [0, 399]),
                                         (129, 1024, 257, [17, 18, 19, 700, 1000, 1023]), (5, 128, 128, []),
-                                        (32, 4096, 4096, [1, 2000, 4000])])
+                                        (32, 4096, 4096, [1, 2000, 4000]),
+                                        (520, 400, 5400, [5, 6, 390])])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_mixed_decomp_gemm_bit_exact(M, K, N, cols, out_dtype):
     X = planted(M, K, cols, seed=3 * M + K)

@@ -104,7 +104,7 @@ def _rand_case(M, N, K, seed):
 
 
 @pytest.mark.parametrize("M,N,K", [(16, 512, 256), (128, 256, 128), (300, 520, 400), (1, 40, 16),
-                                   (257, 1000, 4096), (129, 257, 144)])
+                                   (257, 1000, 4096), (129, 257, 144), (520, 5400, 400), (520, 5000, 144)])
 def test_gemm_int32_accumulator_bit_exact(M, N, K):
     X, Wf, b = _rand_case(M, N, K, M + N + K)
     rq, rS = oracle.quant_per_token(X)
@@ -113,7 +113,10 @@ def test_gemm_int32_accumulator_bit_exact(M, N, K):
     assert_same(host(acc), oracle.gemm_i64(rq, wq).astype(np.int32), "acc")
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 400), (200, 264, 512)])
+# M >= 256 takes the CTA-pair kernel: ragged last row and column tiles, K not a
+# multiple of the 128-byte k-block.
+@pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 400), (200, 264, 512), (520, 5000, 400),
+                                   (520, 5400, 256), (520, 5800, 272)])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_prefill_linear_bit_exact(M, N, K, out_dtype):
     X, Wf, b = _rand_case(M, N, K, 3 * M + N)
