@@ -384,7 +384,7 @@ def bench_decode(args, dev, rank, peaks):
             rows.append({"M": M, "K": DEC_K, "N": N, "us": us, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]})
         del ws
     # static quant alone vs GEMM alone (the C_s / C_g of the PDMIX cost model) at the largest shape
-    return {"workload": "decode: fused static-quant W8A8 linear (quant kernel + PDL-overlapped stream-K GEMM), "
+    return {"workload": "decode: static-quant W8A8 linear in one kernel (quantization fused into the weight-streaming GEMM), "
                         f"rotating weights > L2, CUDA-graph timed", "rows": rows,
             "unit": "GB/s", "peak": peaks["hbm_gbs"], "algorithmic_bytes": "N*K + 8N + 2MK + 2MN per call"}
 

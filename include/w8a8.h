@@ -167,28 +167,36 @@ w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
                               int64_t K, void *out, w8a8_dtype out_dtype, void *workspace,
                               size_t workspace_bytes, void *stream);
 
-/* Bytes of device workspace w8a8_linear_static needs for this shape: M*K
- * bytes rounded up to 256 for the statically quantized activation (no
- * zero-fill needed; every byte read is written by the same call). Calls that
- * overlap on the GPU must not share a workspace. */
+/* Bytes of device workspace w8a8_linear_static needs for this shape: 0 when
+ * it runs as one kernel (M <= 16, or M <= 32 with N <= 4096: the GEMM kernel
+ * quantizes the activation itself), else M*K bytes rounded up to 256 for the
+ * statically quantized activation (no zero-fill needed; every byte read is
+ * written by the same call). Calls that overlap on the GPU must not share a
+ * workspace. */
 size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
- * Decode linear in one call: static per-tensor quantization of bf16 X into
- * the workspace, then the GEMM with the zero-point corrected epilogue. Same
- * result as w8a8_quant_per_tensor followed by w8a8_gemm_dequant with
- * s_x_per_row = 0. For M <= 32 the GEMM kernel is launched with programmatic
- * dependent launch, so it streams the weight while the quantization kernel
- * (and the tail of the kernel before it) runs and reads the quantized
- * activation once that kernel has finished; the rule on writing Wq given for
- * w8a8_gemm_dequant applies.
+ * Decode linear in one call: static per-tensor quantization of bf16 X, then
+ * the GEMM with the zero-point corrected epilogue. Same result as
+ * w8a8_quant_per_tensor followed by w8a8_gemm_dequant with s_x_per_row = 0.
+ * For M <= 16, and for M <= 32 with N <= 4096, it is ONE kernel: the
+ * weight-streaming GEMM loads each bf16 activation k-block and quantizes it in
+ * shared memory before its MMAs read it, and no workspace is used (NULL
+ * allowed). Other shapes quantize into the workspace with a separate kernel
+ * first (every 128-channel tile of the fused kernel re-quantizes the whole
+ * activation, which costs more than it saves there). The Decode-shaped
+ * kernels use programmatic dependent launch like the Decode-shaped
+ * w8a8_gemm_dequant (they stream their first weight tiles while the previous
+ * kernel finishes); the rule on writing Wq given there applies.
  * Source: PDMIX glossary §2.2 (Decode has few tokens and is latency bound, so
  * a per-step quantization launch would be visible overhead) and §2.3 eq.
  * Q_decode; the hardware-acceleration chapter's note that decode is memory
  * bandwidth bound and that runtimes fuse small operations into one kernel.
  *   X            device bf16 [M, K], row stride ldx
  *   S, r, Z      device scalars from w8a8_calibrate_static
- *   Wq, s_w, colsum, bias, out, out_dtype, workspace: as in w8a8_gemm_dequant
+ *   Wq, s_w, colsum, bias, out, out_dtype: as in w8a8_gemm_dequant
+ *   workspace    device, >= w8a8_gemm_workspace_size(M, N, K) bytes, 16-byte
+ *                aligned (NULL allowed when that size is 0)
  */
 w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx, const float *S,
                                const float *r, const int32_t *Z, const int8_t *Wq,
@@ -205,12 +213,13 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
  * latency-critical step that cannot take an allocation's implicit device
  * synchronization. No counterpart on the pages: this is a deployment entry
  * point of this library.
- * The scratch (the quantized activation) is one fixed device array inside
- * the library, 524,288 bytes (32 tokens x 16384), held by every GPU that
- * loads the library until the process exits. It serves M <= 32, N <= 32768
- * and K <= 16384; larger shapes return W8A8_ERR_UNSUPPORTED_SHAPE without
- * launching anything. The call allocates nothing: it launches the same
- * kernels as w8a8_linear_static with the array in place of the workspace.
+ * It always computes in two kernels -- the static quantization into a
+ * scratch, then the Decode-shaped GEMM -- where w8a8_linear_static fuses both
+ * for some shapes; the results are identical. The scratch (the quantized activation) is one fixed device
+ * array inside the library, 524,288 bytes (32 tokens x 16384), held by every
+ * GPU that loads the library until the process exits. It serves M <= 32,
+ * N <= 32768 and K <= 16384; larger shapes return W8A8_ERR_UNSUPPORTED_SHAPE
+ * without launching anything. The call allocates nothing.
  * The first call on a device also sets up that device (looks up the array's
  * device address and zero-fills it once, synchronously): make that first
  * call before any stream capture. All calls on a device share the one array,

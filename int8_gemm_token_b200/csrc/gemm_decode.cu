@@ -70,10 +70,12 @@ constexpr int max_owned_rows() {
   return r;
 }
 
-template <int MP, int SPLIT>
+template <int MP, int SPLIT, bool FUSEQ>
 struct DecCfg {
-  static constexpr int kStageX = MP * kBK;  // int8 activation k-block
-  static constexpr int kStage = kStageW + kStageX;
+  static constexpr int kStageX = MP * kBK;  // int8 activation k-block (128B-swizzled MMA operand)
+  // FUSEQ: the bf16 activation k-block as loaded, two [MP][64] boxes
+  static constexpr int kStageXb = FUSEQ ? 2 * MP * kBK : 0;
+  static constexpr int kStage = kStageW + kStageX + kStageXb;
   // weight rows one CTA finishes, at most (a multiple of 8)
   static constexpr int kR = max_owned_rows<SPLIT>();
   // partial sums this CTA receives from the other SPLIT-1 CTAs of its cluster
@@ -85,7 +87,7 @@ struct DecCfg {
   static constexpr size_t kSmem = static_cast<size_t>(kStages) * kStage + kRedBytes + 1024 + 256;
   static constexpr int kTmemCols = 32;
   static_assert(kR % 8 == 0, "owned rows in 8-row groups");
-  static_assert(kStageX % 1024 == 0, "1 KiB alignment of activation stages");
+  static_assert(kStageX % 1024 == 0 && kStageXb % 1024 == 0, "1 KiB alignment of activation stages");
   static_assert(kStages >= 3, "ring depth");
   static_assert(MP * kR * 4 <= kStages * kStageW, "this CTA's own partial sums fit in the weight ring");
   static_assert(kCtasPerSm * (kSmem + 1024) <= 228 * 1024, "two CTAs per SM");
@@ -192,26 +194,72 @@ __device__ __forceinline__ void epilogue8(const EpilogueArgs &ep, int64_t m, int
   }
 }
 
+constexpr int kQuantThreads = 128;       // FUSEQ: the epilogue warps quantize the activation first
+
+// TMA of one activation k-block into ring slot `slot`: the int8 operand
+// directly (128B swizzle), or with FUSEQ the bf16 k-block as two [MP][64]
+// boxes (no swizzle) for the quantizer warps.
+template <int MP, bool FUSEQ>
+__device__ __forceinline__ void load_activation(const CUtensorMap *tmX, uint64_t *bar, uint8_t *sX, uint8_t *sXb,
+                                                int slot, int32_t kb) {
+  if constexpr (FUSEQ) {
+    uint8_t *dst = sXb + slot * (2 * MP * kBK);
+    tma_load_2d(tmX, bar, dst, kb * kBK, 0);
+    tma_load_2d(tmX, bar, dst + MP * kBK, kb * kBK + kBK / 2, 0);
+  } else {
+    tma_load_2d(tmX, bar, sX + slot * (MP * kBK), kb * kBK, 0);
+  }
+}
+
+// Static per-tensor quantization of one bf16 k-block [MP][128] (two [MP][64]
+// boxes) into the int8 operand layout the MMA reads: K-major, 128-byte rows,
+// the 16-byte chunk c of row m stored at chunk c ^ (m % 8). Thread qt of 128
+// takes the 8-element groups qt, qt + 128, ...: all its loads first, then the
+// arithmetic, then the stores, so the groups overlap; a warp reads 512
+// contiguous bytes per load. Source: PDMIX glossary §2.3 eq. Q_decode,
+// q = clamp(rne(x * r) + Z).
+template <int MP>
+__device__ __forceinline__ void quantize_stage(const uint8_t *xb, uint8_t *xq, int qt, float r, int z) {
+  constexpr int kPer = 2 * MP * 8 / kQuantThreads;  // groups per thread
+  static_assert(kPer * kQuantThreads == 2 * MP * 8, "whole groups per thread");
+  uint4 v[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) v[j] = *reinterpret_cast<const uint4 *>(xb + (qt + j * kQuantThreads) * 16);
+  uint2 q[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) q[j] = quant8_asym_sat(v[j], r, z);
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int g = qt + j * kQuantThreads;
+    const int h = g / (MP * 8);           // box: elements [64 h, 64 h + 64) of the k-block
+    const int m = (g >> 3) - h * MP;      // row
+    const int e = (g & 7) * 8 + h * 64;   // first of the 8 elements within the k-block
+    *reinterpret_cast<uint2 *>(xq + m * kBK + (((e >> 4) ^ (m & 7)) << 4) + (e & 8)) = q[j];
+  }
+}
+
 // Store a 32-bit word to a shared::cluster address (from map_to_rank).
 __device__ __forceinline__ void st_shared_cluster(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-template <int MP, int SPLIT>
+template <int MP, int SPLIT, bool FUSEQ>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     gemm_i8_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                           int64_t M, int64_t N, int64_t K, const __grid_constant__ EpilogueArgs ep,
-                          int32_t *status, uint64_t limit_ns) {
-  using Cfg = DecCfg<MP, SPLIT>;
+                          const float *q_r, const int32_t *q_z, int32_t *status, uint64_t limit_ns) {
+  using Cfg = DecCfg<MP, SPLIT, FUSEQ>;
   constexpr uint32_t kIdesc = idesc_i8(kTileN, MP);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sW = base;                            // kStages x 16 KiB weight ring
-  uint8_t *sX = sW + Cfg::kStages * kStageW;     // kStages x MP*128 activation ring
-  int32_t *sRed = reinterpret_cast<int32_t *>(sX + Cfg::kStages * Cfg::kStageX);  // [SPLIT-1][MP][kR]
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sX + Cfg::kStages * Cfg::kStageX + Cfg::kRedBytes);
+  uint8_t *sX = sW + Cfg::kStages * kStageW;     // kStages x MP*128 int8 activation ring
+  uint8_t *sXb = sX + Cfg::kStages * Cfg::kStageX;  // FUSEQ: kStages x 2*MP*128 bf16 activation ring
+  int32_t *sRed = reinterpret_cast<int32_t *>(sXb + Cfg::kStages * Cfg::kStageXb);  // [SPLIT-1][MP][kR]
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sRed) + Cfg::kRedBytes);
   uint64_t *empty_bar = full_bar + Cfg::kStages;
-  uint64_t *tfull_bar = empty_bar + Cfg::kStages;
+  uint64_t *xq_bar = empty_bar + Cfg::kStages;  // FUSEQ: the int8 operand of a stage is written
+  uint64_t *tfull_bar = xq_bar + Cfg::kStages;
   uint64_t *drain_bar = tfull_bar + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -223,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (int s = 0; s < Cfg::kStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
+      mbar_init(&xq_bar[s], kQuantThreads);
     }
     mbar_init(tfull_bar, 1);
     mbar_init(drain_bar, 1);
@@ -253,14 +302,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       // ---------------------------------------------- TMA producer
       // The first ring of weight tiles does not depend on the previous kernel;
       // the activation may, so its first k-blocks are requested after the wait.
+      constexpr uint32_t kTx = kStageW + (FUSEQ ? Cfg::kStageXb : Cfg::kStageX);
       const int32_t prefetch = nk < Cfg::kStages ? nk : Cfg::kStages;
       for (int32_t i = 0; i < prefetch; ++i) {  // the ring starts empty: no waits
-        mbar_arrive_expect_tx(&full_bar[i], kStageW + Cfg::kStageX);
+        mbar_arrive_expect_tx(&full_bar[i], kTx);
         tma_load_2d(&tmW, &full_bar[i], sW + i * kStageW, (kb0 + i) * kBK, wrow);
       }
       pdl_wait_prerequisite();
-      for (int32_t i = 0; i < prefetch; ++i)
-        tma_load_2d(&tmX, &full_bar[i], sX + i * Cfg::kStageX, (kb0 + i) * kBK, 0);
+      for (int32_t i = 0; i < prefetch; ++i) load_activation<MP, FUSEQ>(&tmX, &full_bar[i], sX, sXb, i, kb0 + i);
       int stage = prefetch % Cfg::kStages;
       uint32_t phase = prefetch == Cfg::kStages ? 1u : 0u;
       // parity of the last fill of every stage, to wait for copies in flight on failure
@@ -271,9 +320,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&full_bar[stage], kStageW + Cfg::kStageX);
+        mbar_arrive_expect_tx(&full_bar[stage], kTx);
         tma_load_2d(&tmW, &full_bar[stage], sW + stage * kStageW, (kb0 + i) * kBK, wrow);
-        tma_load_2d(&tmX, &full_bar[stage], sX + stage * Cfg::kStageX, (kb0 + i) * kBK, 0);
+        load_activation<MP, FUSEQ>(&tmX, &full_bar[stage], sX, sXb, stage, kb0 + i);
         issued_mask |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == Cfg::kStages) {
@@ -297,7 +346,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       uint32_t phase = 0;
       bool ok = true;
       for (int32_t i = 0; i < nk; ++i) {
-        if (!mbar_wait_bounded(&full_bar[stage], phase, abort_flag, limit_ns)) {
+        if (!mbar_wait_bounded(&full_bar[stage], phase, abort_flag, limit_ns) ||
+            (FUSEQ && !mbar_wait_bounded(&xq_bar[stage], phase, abort_flag, limit_ns))) {
           ok = false;
           break;
         }
@@ -321,6 +371,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         mbar_wait_bounded(drain_bar, 0, nullptr, limit_ns / 16 + 1);
       } else {
         mma_commit(tfull_bar);
+      }
+    }
+  }
+
+  if (FUSEQ && warp >= kEpiWarp0) {
+    // ------------------------------------------------ activation quantizers (FUSEQ)
+    // Per stage: the bf16 k-block [MP][128] -> the int8 operand, fenced for
+    // the tensor core, then xq_bar. The epilogue warps are idle until tfull.
+    pdl_wait_prerequisite();  // r and Z may be written by the previous kernel
+    const float r = __ldg(q_r);
+    const int z = __ldg(q_z);
+    const int qt = threadIdx.x - kEpiWarp0 * 32;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int32_t i = 0; i < nk; ++i) {
+      if (!mbar_wait_bounded(&full_bar[stage], phase, abort_flag, limit_ns)) {
+        record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      quantize_stage<MP>(sXb + stage * Cfg::kStageXb, sX + stage * Cfg::kStageX, qt, r, z);
+      fence_proxy_async_smem();
+      mbar_arrive(&xq_bar[stage]);
+      if (++stage == Cfg::kStages) {
+        stage = 0;
+        phase ^= 1u;
       }
     }
   }
@@ -427,28 +503,40 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 // Dynamic shared memory of the kernel, and the largest shared-memory carveout:
 // without it the driver may size the carveout for one CTA per SM.
-template <int MP, int SPLIT>
+template <int MP, int SPLIT, bool FUSEQ>
 cudaError_t configure_decode_kernel() {
-  auto kern = gemm_i8_decode_kernel<MP, SPLIT>;
+  auto kern = gemm_i8_decode_kernel<MP, SPLIT, FUSEQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(DecCfg<MP, SPLIT>::kSmem));
+                                       static_cast<int>(DecCfg<MP, SPLIT, FUSEQ>::kSmem));
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
 }
 
-template <int MP, int SPLIT>
-cudaError_t launch_decode_t(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
+// The activation operand: int8 Xq [M, K] (row stride ldx bytes) or, with
+// FUSEQ, bf16 X [M, K] (row stride ldx elements) with the static r and Z.
+struct DecodeActivation {
+  const void *x;
+  int64_t ldx;
+  const float *r;
+  const int32_t *z;
+};
+
+template <int MP, int SPLIT, bool FUSEQ>
+cudaError_t launch_decode_t(const DecodeActivation &act, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                             const EpilogueArgs &ep, int32_t *status, cudaStream_t s) {
-  using Cfg = DecCfg<MP, SPLIT>;
+  using Cfg = DecCfg<MP, SPLIT, FUSEQ>;
   alignas(64) CUtensorMap tmW, tmX;
   if (!encode_tmap_2d(&tmW, Wq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                       static_cast<uint64_t>(K), kBK, kTileN, true))
     return cudaErrorInvalidValue;
-  if (!encode_tmap_2d(&tmX, Xq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                      static_cast<uint64_t>(ldx), kBK, MP, true))
-    return cudaErrorInvalidValue;
-  auto kern = gemm_i8_decode_kernel<MP, SPLIT>;
-  cudaError_t e = configure_decode_kernel<MP, SPLIT>();
+  const bool ok_x = FUSEQ ? encode_tmap_2d(&tmX, act.x, TmapType::kBF16, static_cast<uint64_t>(K),
+                                           static_cast<uint64_t>(M), static_cast<uint64_t>(act.ldx) * 2, kBK / 2,
+                                           MP, false)
+                          : encode_tmap_2d(&tmX, act.x, TmapType::kU8, static_cast<uint64_t>(K),
+                                           static_cast<uint64_t>(M), static_cast<uint64_t>(act.ldx), kBK, MP, true);
+  if (!ok_x) return cudaErrorInvalidValue;
+  auto kern = gemm_i8_decode_kernel<MP, SPLIT, FUSEQ>;
+  cudaError_t e = configure_decode_kernel<MP, SPLIT, FUSEQ>();
   if (e != cudaSuccess) return e;
   const int64_t tiles = (N + kTileN - 1) / kTileN;
   cudaLaunchConfig_t cfg = {};
@@ -465,7 +553,7 @@ cudaError_t launch_decode_t(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, M, N, K, ep, status, kWaitLimitNs);
+  return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, M, N, K, ep, act.r, act.z, status, kWaitLimitNs);
 }
 
 // A kernel with the decode kernel's launch shape and no body. The runtime's
@@ -477,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_occupancy_standin
 
 // Clusters of SPLIT decode CTAs that can be resident at once on the current
 // device (cached per device).
-template <int MP, int SPLIT>
+template <int MP, int SPLIT, bool FUSEQ>
 int max_active_clusters() {
   constexpr int kMaxDevices = 64;
   static std::atomic<int> cache[kMaxDevices];
@@ -488,7 +576,7 @@ int max_active_clusters() {
   }
   int n = cache[dev].load(std::memory_order_relaxed);
   if (n > 0) return n;
-  using Cfg = DecCfg<MP, SPLIT>;
+  using Cfg = DecCfg<MP, SPLIT, FUSEQ>;
   if (cudaFuncSetAttribute(decode_occupancy_standin, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            200 * 1024) != cudaSuccess ||
       cudaFuncSetAttribute(decode_occupancy_standin, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -515,56 +603,66 @@ int max_active_clusters() {
   return n;
 }
 
-template <int MP>
+template <int MP, bool FUSEQ>
 int max_active_clusters_of(int split) {
   switch (split) {
-    case 8: return max_active_clusters<MP, 8>();
-    case 7: return max_active_clusters<MP, 7>();
-    case 6: return max_active_clusters<MP, 6>();
-    case 5: return max_active_clusters<MP, 5>();
-    case 4: return max_active_clusters<MP, 4>();
-    case 3: return max_active_clusters<MP, 3>();
-    case 2: return max_active_clusters<MP, 2>();
-    default: return max_active_clusters<MP, 1>();
+    case 8: return max_active_clusters<MP, 8, FUSEQ>();
+    case 7: return max_active_clusters<MP, 7, FUSEQ>();
+    case 6: return max_active_clusters<MP, 6, FUSEQ>();
+    case 5: return max_active_clusters<MP, 5, FUSEQ>();
+    case 4: return max_active_clusters<MP, 4, FUSEQ>();
+    case 3: return max_active_clusters<MP, 3, FUSEQ>();
+    case 2: return max_active_clusters<MP, 2, FUSEQ>();
+    default: return max_active_clusters<MP, 1, FUSEQ>();
   }
 }
 
 // Largest cluster size (1..8) whose clusters, one per 128-row tile, are all
 // resident at once, with at least 2 k-blocks per CTA.
-template <int MP>
+template <int MP, bool FUSEQ>
 int decode_split_mp(int64_t N, int64_t K) {
   const int64_t tiles = (N + kTileN - 1) / kTileN;
   const int64_t nkb = (K + kBK - 1) / kBK;
   for (int s = kMaxSplit; s >= 2; --s)
-    if (nkb >= 2 * s && tiles <= max_active_clusters_of<MP>(s)) return s;
+    if (nkb >= 2 * s && tiles <= max_active_clusters_of<MP, FUSEQ>(s)) return s;
   return 1;
 }
 
-template <int MP>
-cudaError_t launch_decode_mp(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
+template <int MP, bool FUSEQ>
+cudaError_t launch_decode_mp(const DecodeActivation &act, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                              const EpilogueArgs &ep, int32_t *status, cudaStream_t s) {
-  switch (decode_split_mp<MP>(N, K)) {
-    case 8: return launch_decode_t<MP, 8>(Xq, ldx, Wq, M, N, K, ep, status, s);
-    case 7: return launch_decode_t<MP, 7>(Xq, ldx, Wq, M, N, K, ep, status, s);
-    case 6: return launch_decode_t<MP, 6>(Xq, ldx, Wq, M, N, K, ep, status, s);
-    case 5: return launch_decode_t<MP, 5>(Xq, ldx, Wq, M, N, K, ep, status, s);
-    case 4: return launch_decode_t<MP, 4>(Xq, ldx, Wq, M, N, K, ep, status, s);
-    case 3: return launch_decode_t<MP, 3>(Xq, ldx, Wq, M, N, K, ep, status, s);
-    case 2: return launch_decode_t<MP, 2>(Xq, ldx, Wq, M, N, K, ep, status, s);
-    default: return launch_decode_t<MP, 1>(Xq, ldx, Wq, M, N, K, ep, status, s);
+  switch (decode_split_mp<MP, FUSEQ>(N, K)) {
+    case 8: return launch_decode_t<MP, 8, FUSEQ>(act, Wq, M, N, K, ep, status, s);
+    case 7: return launch_decode_t<MP, 7, FUSEQ>(act, Wq, M, N, K, ep, status, s);
+    case 6: return launch_decode_t<MP, 6, FUSEQ>(act, Wq, M, N, K, ep, status, s);
+    case 5: return launch_decode_t<MP, 5, FUSEQ>(act, Wq, M, N, K, ep, status, s);
+    case 4: return launch_decode_t<MP, 4, FUSEQ>(act, Wq, M, N, K, ep, status, s);
+    case 3: return launch_decode_t<MP, 3, FUSEQ>(act, Wq, M, N, K, ep, status, s);
+    case 2: return launch_decode_t<MP, 2, FUSEQ>(act, Wq, M, N, K, ep, status, s);
+    default: return launch_decode_t<MP, 1, FUSEQ>(act, Wq, M, N, K, ep, status, s);
   }
 }
 
 }  // namespace
 
-int decode_split(int64_t M, int64_t N, int64_t K) {
-  return M <= 16 ? decode_split_mp<16>(N, K) : decode_split_mp<32>(N, K);
+int decode_split(int64_t M, int64_t N, int64_t K, bool fused_quant) {
+  if (fused_quant) return M <= 16 ? decode_split_mp<16, true>(N, K) : decode_split_mp<32, true>(N, K);
+  return M <= 16 ? decode_split_mp<16, false>(N, K) : decode_split_mp<32, false>(N, K);
 }
 
 cudaError_t launch_gemm_decode(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                                const EpilogueArgs &ep, int32_t *status, cudaStream_t s) {
-  if (M <= 16) return launch_decode_mp<16>(Xq, ldx, Wq, M, N, K, ep, status, s);
-  return launch_decode_mp<32>(Xq, ldx, Wq, M, N, K, ep, status, s);
+  const DecodeActivation act{Xq, ldx, nullptr, nullptr};
+  if (M <= 16) return launch_decode_mp<16, false>(act, Wq, M, N, K, ep, status, s);
+  return launch_decode_mp<32, false>(act, Wq, M, N, K, ep, status, s);
+}
+
+cudaError_t launch_linear_static_decode(const uint16_t *X, int64_t ldx, const float *r, const int32_t *Z,
+                                        const int8_t *Wq, int64_t M, int64_t N, int64_t K, const EpilogueArgs &ep,
+                                        int32_t *status, cudaStream_t s) {
+  const DecodeActivation act{X, ldx, r, Z};
+  if (M <= 16) return launch_decode_mp<16, true>(act, Wq, M, N, K, ep, status, s);
+  return launch_decode_mp<32, true>(act, Wq, M, N, K, ep, status, s);
 }
 
 }  // namespace w8a8

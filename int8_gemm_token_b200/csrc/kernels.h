@@ -60,8 +60,14 @@ cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_
 // dependents launch early must not write Wq).
 cudaError_t launch_gemm_decode(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                                const EpilogueArgs &ep, int32_t *status, cudaStream_t s);
+// The Decode linear in one kernel: the same GEMM, with the static per-tensor
+// quantization of bf16 X (row stride ldx elements, device scalars r and Z)
+// done inside it on each activation k-block before the MMAs read it.
+cudaError_t launch_linear_static_decode(const uint16_t *X, int64_t ldx, const float *r, const int32_t *Z,
+                                        const int8_t *Wq, int64_t M, int64_t N, int64_t K, const EpilogueArgs &ep,
+                                        int32_t *status, cudaStream_t s);
 // Cluster size the decode GEMM uses for this shape on the current device.
-int decode_split(int64_t M, int64_t N, int64_t K);
+int decode_split(int64_t M, int64_t N, int64_t K, bool fused_quant);
 
 // LLM.int8() outlier split: column-flag pass into a K-bit bitmap in
 // `workspace` (outlier_workspace_bytes(K); zeroed by the launcher), then the

@@ -9,7 +9,9 @@
 // This entry point needs no memory from them: its scratch (the statically
 // quantized activation handed from the quantization kernel to the GEMM)
 // lives in one file-scope device array of fixed size, which every GPU that
-// loads the library holds until the process exits.
+// loads the library holds until the process exits. It runs the two-kernel
+// form of the Decode linear (quantization, then the decode GEMM), which gives
+// the same result as the fused kernel of w8a8_linear_static.
 #include <mutex>
 
 #include "device.cuh"

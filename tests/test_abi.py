@@ -72,7 +72,9 @@ def test_gemm_host_checks(L):
 def test_linear_static_workspace_check(L):
     f = L.w8a8_linear_static
     # X, M, K, ldx, S, r, Z, Wq, s_w, colsum, bias, N, out, dt, ws, wsb, stream
-    assert f(GOOD, 4, 64, 64, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, None, 8, GOOD, 0, None, 0, None) == 9
+    # more than 32 tokens: the quantized activation needs M*K bytes of workspace
+    assert f(GOOD, 40, 64, 64, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, None, 8, GOOD, 0, None, 0, None) == 9
+    assert f(GOOD, 40, 64, 64, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, None, 8, GOOD, 0, GOOD, 40 * 64 - 1, None) == 9
     assert f(GOOD, 4, 64, 64, GOOD, GOOD, None, GOOD, GOOD, GOOD, None, 8, GOOD, 0, GOOD, 4096, None) == 1
 
 
@@ -102,5 +104,8 @@ def test_valid_call_without_a_gpu_reports_no_device(L):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert L.w8a8_quant_per_token(GOOD, 4, 32, 32, GOOD, GOOD, None) == 10
-    assert w8a8.w8a8_gemm_workspace_size(4, 8, 64) >= 4 * 64
+    assert w8a8.w8a8_gemm_workspace_size(4, 8, 64) == 0  # one kernel: quantized inside the GEMM
+    assert w8a8.w8a8_gemm_workspace_size(32, 4096, 64) == 0
+    assert w8a8.w8a8_gemm_workspace_size(32, 4104, 64) >= 32 * 64  # quantization kernel first
+    assert w8a8.w8a8_gemm_workspace_size(64, 8, 64) >= 64 * 64
     assert w8a8.lib().int8_outlier_split_workspace_size(8192) >= 8192 // 8

@@ -299,3 +299,44 @@ def test_decode_back_to_back_calls_overlap_safely(graph):
     for (X, S, r, Z, Wq, s_w, cs, Xq_in, out_a, out_b), ref in zip(layers, refs):
         assert_same(host_bf16(out_a), ref, "linear_static")
         assert_same(host_bf16(out_b), ref, "gemm_dequant")
+
+
+def _all_finite_bf16(rows):
+    """Every finite bf16 bit pattern (65,280 of them) as [rows, K], K the next
+    multiple of 16, the tail padded with +0."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    bits = bits[(bits & 0x7F80) != 0x7F80]
+    K = -(-bits.size // rows // 16) * 16
+    out = np.zeros(rows * K, dtype=np.uint16)
+    out[:bits.size] = bits
+    return out.reshape(rows, K)
+
+
+@pytest.mark.parametrize("r,Z", [(1.0, 0), (0.013, -128), (127.0 / 3.5, 7), (1e-30, 127), (3.0e38, -5),
+                                 (1000.0, -17)])
+def test_quant_per_tensor_every_finite_bf16_value(r, Z):
+    """q = clamp(rne(x * r) + Z, -128, 127) for every finite bf16 x: ties to
+    even, values that overflow x * r, subnormals and signed zeros."""
+    X = _all_finite_bf16(510)
+    rd = torch.tensor([r], dtype=torch.float32, device="cuda")
+    Zd = torch.tensor([Z], dtype=torch.int32, device="cuda")
+    got = host(W.w8a8_quant_per_tensor(dev_bf16(X), rd, Zd))
+    assert_same(got, oracle.quant_per_tensor(X, np.float32(r), Z), "Xq")
+
+
+@pytest.mark.parametrize("M,N", [(32, 1000), (16, 1000), (24, 5000)])
+def test_decode_linear_static_every_finite_bf16_activation(M, N):
+    """Feed the Decode linear every finite bf16 value as its activation (rows
+    of K = 2048, 4080 or 2720) and compare the outputs with the oracle's
+    quantize -> GEMM -> epilogue: the first two shapes quantize inside the GEMM
+    kernel, the third with the separate quantization kernel."""
+    X = _all_finite_bf16(M)
+    K = X.shape[1]
+    case = synth.decode_static(M=M, N=N, K=K, seed=5)
+    S, r, Z = W.w8a8_calibrate_static(dev_bf16(case.Xcal))
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(case.W))
+    out = W.w8a8_linear_static(dev_bf16(X), S, r, Z, Wq, s_w, cs, out_dtype=torch.float32)
+    rS, rr, rZ = oracle.calibrate_static(case.Xcal)
+    rwq, rws, rwc = oracle.quant_weight_per_channel(case.W)
+    _, _, y = oracle.linear_decode(X, rr, rZ, rS, rwq, rws, rwc)
+    assert_same(host(out), y, "out")
