@@ -57,6 +57,33 @@ def load_peaks():
 # INT8 dense tensor throughput is twice bf16 on B200 (4.5 vs 2.25 PFLOP/s nominal)
 INT8_OVER_BF16 = 2.0
 
+# DRAM traffic of one launch of the prefill GEMM kernel at this workload, from
+# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum; the summary
+# with its command is profiles/gemm_i8_tc2_prefill_7b_2048x4096x11008.txt).
+# It describes the kernel built from these sources only: once they change, the
+# bench reports no traffic until the kernel is profiled again.
+TC2_TRAFFIC = {
+    "bytes": 53_672_192 + 6_080_512,
+    "sources": ["int8_gemm_token_b200/csrc/gemm_tc.cu", "int8_gemm_token_b200/csrc/device.cuh",
+                "int8_gemm_token_b200/csrc/kernels.h"],
+    "sources_sha256": "fac04883a3cab040e44000a5424d4e02b8458dbd3f8e20b0fb1c1aff05f8a49d",
+    "profile": "profiles/gemm_i8_tc2_prefill_7b_2048x4096x11008.txt",
+}
+
+
+def profiled_traffic(entry):
+    """The recorded per-launch DRAM bytes if the kernel's sources are unchanged, else None."""
+    import hashlib
+    root = os.path.dirname(os.path.abspath(__file__))
+    h = hashlib.sha256()
+    try:
+        for f in entry["sources"]:
+            with open(os.path.join(root, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return entry["bytes"] if h.hexdigest() == entry["sources_sha256"] else None
+
 
 class ClockSampler:
     """Samples SM clock and clock-event reasons with NVML while running."""
@@ -306,10 +333,12 @@ def run_ours(args, world, rank, local):
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "parallelism": f"replicas x{world}",
                        "l2": f"{N_SETS} rotating X/Wq/out sets, {N_SETS * 115} MB > 126 MB L2"},
-            "roofline": {"bound": "tensor", "kernel": "gemm_i8_tc_kernel", "achieved": gemm_tops,
+            "roofline": {"bound": "tensor", "kernel": "gemm_i8_tc2_kernel", "achieved": gemm_tops,
                          "peak": int8_peak, "unit": "TOPS", "frac": gemm_tops / int8_peak,
                          "peak_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (int8/bf16 nominal)",
-                         "traffic": None},
+                         "traffic": profiled_traffic(TC2_TRAFFIC), "traffic_unit": "B per launch",
+                         "traffic_profile": TC2_TRAFFIC["profile"],
+                         "algorithmic_bytes": M * K + N * K + 2 * M * N + 4 * M + 8 * N},
             "quant": {"kernel": "quant_per_token_kernel", "ms": quant_ms, "achieved": quant_gbs,
                       "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": quant_gbs / peaks["hbm_gbs"],
                       "C_s_over_C_g": quant_ms / gemm_ms},

@@ -60,3 +60,13 @@ def test_reference_arm_runs_on_rank_zero_only():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                           "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_profiled_traffic_only_for_unchanged_kernel_sources():
+    import bench
+    entry = dict(bench.TC2_TRAFFIC)
+    assert bench.profiled_traffic(entry) == entry["bytes"]
+    stale = dict(entry, sources_sha256="0" * 64)
+    assert bench.profiled_traffic(stale) is None
+    missing = dict(entry, sources=["no/such/file.cu"])
+    assert bench.profiled_traffic(missing) is None
