@@ -220,6 +220,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     peaks = load_peaks()
     int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    int8_sustained = (peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]) * INT8_OVER_BF16
 
     def bf16_dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -254,23 +255,37 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
 
     # ---------------------------------------------------------------- timed
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # The steps run back to back with events only at both ends: the kernels
+    # use programmatic dependent launch, so each one starts under the tail of
+    # the one before, and an event recorded between two kernels would stop that.
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
+        t0.record(stream)
         for i in range(args.steps):
-            s = sets[i % N_SETS]
-            ev[i][0].record(stream)
-            W.w8a8_quant_per_token(s["X"], Xq=s["Xq"], S_x=s["S"], stream=stream)
-            ev[i][1].record(stream)
-            W.w8a8_gemm_dequant(s["Xq"], s["S"], s["Wq"], s["s_w"], bias=s["bias"], out=s["out"], stream=stream)
-            ev[i][2].record(stream)
+            step(sets[i % N_SETS])
+        t1.record(stream)
         torch.cuda.synchronize()
     barrier()
-    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    total_ms = t0.elapsed_time(t1)
+    ms_per_step = max_ranks(total_ms / args.steps)
+    # Per-kernel durations (roofline, quant row): a second timed pass with
+    # events around each kernel, which serialises them.
+    n_bd = max(3, min(args.steps, 200))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_bd)]
+    torch.cuda.synchronize()
+    for i in range(n_bd):
+        s = sets[i % N_SETS]
+        ev[i][0].record(stream)
+        W.w8a8_quant_per_token(s["X"], Xq=s["Xq"], S_x=s["S"], stream=stream)
+        ev[i][1].record(stream)
+        W.w8a8_gemm_dequant(s["Xq"], s["S"], s["Wq"], s["s_w"], bias=s["bias"], out=s["out"], stream=stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
     quant_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     gemm_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    ms_per_step = max_ranks(total_ms / args.steps)
     ops = 2.0 * M * N * K
     value = whole_job_tops(ops, world, ms_per_step)
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
@@ -334,8 +349,10 @@ def run_ours(args, world, rank, local):
             "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "parallelism": f"replicas x{world}",
                        "l2": f"{N_SETS} rotating X/Wq/out sets, {N_SETS * 115} MB > 126 MB L2"},
             "roofline": {"bound": "tensor", "kernel": "gemm_i8_tc2_kernel", "achieved": gemm_tops,
-                         "peak": int8_peak, "unit": "TOPS", "frac": gemm_tops / int8_peak,
-                         "peak_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (int8/bf16 nominal)",
+                         "peak": int8_sustained, "unit": "TOPS", "frac": gemm_tops / int8_sustained,
+                         "peak_source": f"{peaks['source']} sustained bf16 {peaks['bf16_tflops_sustained']} TFLOP/s x 2 "
+                                        "(int8/bf16 nominal); the kernel is timed right after the K-step loop",
+                         "frac_of_burst_peak": gemm_tops / int8_peak,
                          "traffic": profiled_traffic(TC2_TRAFFIC), "traffic_unit": "B per launch",
                          "traffic_profile": TC2_TRAFFIC["profile"],
                          "algorithmic_bytes": M * K + N * K + 2 * M * N + 4 * M + 8 * N},
@@ -349,6 +366,10 @@ def run_ours(args, world, rank, local):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 2 * args.steps,
+            "timing": {"value": "K back-to-back steps between two CUDA events (kernels overlap through "
+                                "programmatic dependent launch)",
+                       "per_kernel": f"{n_bd} further steps with events around each kernel (serialised); "
+                                     "roofline.achieved and quant use these"},
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -413,8 +434,9 @@ def bench_decode(args, dev, rank, peaks):
             rows.append({"M": M, "K": DEC_K, "N": N, "us": us, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]})
         del ws
     # static quant alone vs GEMM alone (the C_s / C_g of the PDMIX cost model) at the largest shape
-    return {"workload": "decode: static-quant W8A8 linear in one kernel (quantization fused into the weight-streaming GEMM), "
-                        f"rotating weights > L2, CUDA-graph timed", "rows": rows,
+    return {"workload": "decode: static-quant W8A8 linear, w8a8_linear_static (one kernel with the quantization fused "
+                        "into the weight-streaming GEMM for M <= 16 or N <= 4096, else quantization kernel + GEMM), "
+                        "back-to-back calls, rotating weights > L2, CUDA-graph timed", "rows": rows,
             "unit": "GB/s", "peak": peaks["hbm_gbs"], "algorithmic_bytes": "N*K + 8N + 2MK + 2MN per call"}
 
 
@@ -495,6 +517,18 @@ def bench_block(args, dev, rank, peaks, int8_peak):
             q_ms += sum(e[0].elapsed_time(e[1]) for e in evs) / reps
             g_ms += sum(e[1].elapsed_time(e[2]) for e in evs) / reps
     prefill_ops = sum(2.0 * 4096 * Ly["K"] * Ly["N"] for Ly in layers)
+    # the whole Prefill pass back to back (events only at both ends, so the
+    # kernels overlap through programmatic dependent launch)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for rep in range(reps):
+        for Ly in layers:
+            W.w8a8_quant_per_token(Ly["Xp"], Xq=Ly["Xq"], S_x=Ly["Sx"])
+            W.w8a8_gemm_dequant(Ly["Xq"], Ly["Sx"], Ly["Wq"], Ly["s_w"], out=Ly["outp"])
+    b.record(stream)
+    torch.cuda.synchronize()
+    pass_ms = a.elapsed_time(b) / reps
 
     def decode_all(step):
         for Ly in layers:
@@ -507,7 +541,8 @@ def bench_block(args, dev, rank, peaks, int8_peak):
     assert W.w8a8_check_device_error() == 0
     return {"workload": "PDMIX block: QKV 4096->12288, O 4096->4096, gate+up 4096->22016, down 11008->4096; "
                         "prefill 4096 tokens, then 64 decode steps x 32 tokens",
-            "prefill_us": (q_ms + g_ms) * 1e3, "prefill_TOPS": prefill_ops / ((q_ms + g_ms) * 1e-3) / 1e12,
+            "prefill_us": pass_ms * 1e3, "prefill_TOPS": prefill_ops / (pass_ms * 1e-3) / 1e12,
+            "prefill_kernels_serialised_us": (q_ms + g_ms) * 1e3,
             "prefill_gemm_frac_int8": prefill_ops / (g_ms * 1e-3) / 1e12 / int8_peak,
             "prefill_C_s_over_C_g": q_ms / g_ms,
             "decode_total_us": 64 * step_us, "decode_step_us": step_us,

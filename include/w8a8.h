@@ -153,11 +153,12 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
  * 8 CTAs per 128 output channels splits K, and the partial int32 sums are
  * added in distributed shared memory, so the call keeps no state in device
  * memory between calls and calls on different streams may overlap.
- * That kernel uses programmatic dependent launch: it may start while the
- * previous kernel on the stream is still running, and it begins streaming Wq
- * at once. Everything else (Xq, S_x, Z, colsum, s_w, bias, out) is touched
- * only after the previous kernel has completed. So Wq, a constant weight,
- * must not be written by a kernel that lets its dependents launch early
+ * Every GEMM kernel of this call (Decode-shaped or not) uses programmatic
+ * dependent launch: it may start while the previous kernel on the stream is
+ * still running, and it loads its first weight tiles at once. Everything
+ * else (Xq, S_x, Z, colsum, s_w, bias, out) is touched only after the
+ * previous kernel has completed. So Wq, a constant weight, must not be
+ * written by a kernel that lets its dependents launch early
  * (griddepcontrol.launch_dependents) and immediately precedes this call; no
  * kernel of this library that writes Wq does so.
  */

@@ -306,7 +306,7 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
   }
   int8_t *Xq = static_cast<int8_t *>(workspace);
   cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq,
-                                          d->sm_count, st);
+                                          d->sm_count, st, /*pdl=*/true);
   if (e != cudaSuccess) return W8A8_ERR_CUDA;
   return from_cuda(launch_gemm_tc(Xq, Wq, M, N, K, ep, false, d->sm_count, d->status, st));
 }

@@ -216,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncwarp();  // bar.sync is warp-aligned: reconverge after the single-thread set-up
   __syncthreads();
   tc_fence_after();
+  pdl_launch_dependents();
   const uint32_t tmem_base = *tmem_slot;
 
   const int64_t num_m = (M + kBM - 1) / kBM;
@@ -226,14 +227,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued_mask = 0, issued_parity = 0;
+      // The first ring of weight tiles does not depend on the previous kernel
+      // in the stream; the activation may, so its tiles follow the wait.
+      int pre = 0;
+      if (blockIdx.x < num_tiles) {
+        pre = nkb < STAGES ? nkb : STAGES;
+        const int32_t nrow0 = static_cast<int32_t>((blockIdx.x / num_m) * BN);
+        for (int kb = 0; kb < pre; ++kb) {  // the ring starts empty: no waits
+          mbar_arrive_expect_tx(&full_bar[kb], kStageA + Cfg::kStageB);
+          tma_load_2d(&tmB, &full_bar[kb], sB + kb * Cfg::kStageB, kb * kBK, nrow0);
+        }
+      }
+      pdl_wait_prerequisite();
+      if (pre > 0) {
+        const int32_t mrow0 = static_cast<int32_t>((blockIdx.x % num_m) * kBM);
+        for (int kb = 0; kb < pre; ++kb) tma_load_2d(&tmA, &full_bar[kb], sA + kb * kStageA, kb * kBK, mrow0);
+      }
+      int stage = pre % STAGES;
+      uint32_t phase = pre == STAGES ? 1u : 0u;
+      uint32_t issued_mask = pre >= 32 ? 0xFFFFFFFFu : ((1u << pre) - 1u), issued_parity = 0;
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int32_t mrow = static_cast<int32_t>((tile % num_m) * kBM);
         const int32_t nrow = static_cast<int32_t>((tile / num_m) * BN);
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = tile == blockIdx.x ? pre : 0; kb < nkb; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag, limit_ns)) {
             ok = false;
             break;
@@ -261,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
+      pdl_wait_prerequisite();  // bounded waits below count from here, not from an early launch
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -307,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= kEpiWarp0) {
+    pdl_wait_prerequisite();  // S_x, scales, side inputs and `out` belong to the previous kernel until then
     // -------------------------------------------------- epilogue
     const int q = warp - kEpiWarp0;  // TMEM lane quarter of this warp (warp % 4)
     const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
@@ -420,6 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
+  pdl_launch_dependents();
   const uint32_t tmem_base = *tmem_slot;
 
   const int64_t num_m = (M + kTileM - 1) / kTileM;
@@ -432,13 +452,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer (both CTAs)
-      int stage = 0;
-      uint32_t phase = 0;
+      // The first ring of weight tiles does not depend on the previous kernel
+      // in the stream; the activation may, so its tiles follow the wait.
+      int pre = 0;
+      if (cluster_id < num_tiles) {
+        pre = nkb < STAGES ? nkb : STAGES;
+        const int32_t brow0 = static_cast<int32_t>((cluster_id / num_m) * kTileN + rank * kHalf);
+        for (int kb = 0; kb < pre; ++kb) {  // the ring starts empty: no waits
+          if (leader) mbar_arrive_expect_tx(&full_bar[kb], 2 * (kStageA2 + kStageB2));
+          tma_load_2d_pair(&tmB, map_to_rank(&full_bar[kb], 0), sB + kb * kStageB2, kb * kBK, brow0);
+        }
+      }
+      pdl_wait_prerequisite();
+      if (pre > 0) {
+        const int32_t arow0 = static_cast<int32_t>((cluster_id % num_m) * kTileM + rank * kHalf);
+        for (int kb = 0; kb < pre; ++kb)
+          tma_load_2d_pair(&tmA, map_to_rank(&full_bar[kb], 0), sA + kb * kStageA2, kb * kBK, arow0);
+      }
+      int stage = pre % STAGES;
+      uint32_t phase = pre == STAGES ? 1u : 0u;
       bool ok = true;
       for (int64_t tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
         const int32_t arow = static_cast<int32_t>((tile % num_m) * kTileM + rank * kHalf);
         const int32_t brow = static_cast<int32_t>((tile / num_m) * kTileN + rank * kHalf);
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = tile == cluster_id ? pre : 0; kb < nkb; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag, limit_ns)) {
             ok = false;
             break;
@@ -461,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------ pair MMA issuer (leader)
+      pdl_wait_prerequisite();  // bounded waits below count from here, not from an early launch
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -508,6 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= kEpiWarp0) {
+    pdl_wait_prerequisite();  // S_x, scales, side inputs and `out` belong to the previous kernel until then
     // -------------------------------------------------- epilogue (both CTAs)
     const int q = warp - kEpiWarp0;
     const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
@@ -583,13 +622,15 @@ cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t 
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, M, N, K, ep, status, kWaitLimitNs);
 }
 
@@ -610,9 +651,17 @@ cudaError_t launch_tc_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N
                                        static_cast<int>(Cfg::kSmem));
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
-  const unsigned grid = static_cast<unsigned>(tiles < num_sms ? tiles : num_sms);
-  kern<<<grid, kThreads, Cfg::kSmem, s>>>(tmA, tmB, M, N, K, ep, status, kWaitLimitNs);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles < num_sms ? tiles : num_sms));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, M, N, K, ep, status, kWaitLimitNs);
 }
 
 }  // namespace

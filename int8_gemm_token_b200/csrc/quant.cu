@@ -37,6 +37,12 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__
   const int64_t chunks = K >> 3;
   const bool row_ok = m < M;
   const uint16_t *xrow = X + m * ldx;
+  // Launched with programmatic stream serialization, this kernel may start
+  // while the previous kernel still runs: let the dependent GEMM launch (it
+  // touches nothing this kernel writes before its own wait), then wait for the
+  // previous kernel before reading X or writing Xq, S_x.
+  pdl_launch_dependents();
+  pdl_wait_prerequisite();
 
   uint4 v[VPT];
   uint32_t m2 = 0;
@@ -77,9 +83,16 @@ static cudaError_t launch_per_token_t(const uint16_t *X, int64_t M, int64_t K, i
                                       int8_t *Xq, float *S_x, cudaStream_t s) {
   constexpr int NT = G == 32 ? 128 : 256;
   constexpr int R = NT / G;
-  const unsigned blocks = static_cast<unsigned>((M + R - 1) / R);
-  quant_per_token_kernel<G, VPT><<<blocks, NT, 0, s>>>(X, M, K, ldx, Xq, S_x);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((M + R - 1) / R));
+  cfg.blockDim = dim3(NT);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quant_per_token_kernel<G, VPT>, X, M, K, ldx, Xq, S_x);
 }
 
 cudaError_t launch_quant_per_token(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,

@@ -63,10 +63,16 @@ def test_reference_arm_runs_on_rank_zero_only():
 
 
 def test_profiled_traffic_only_for_unchanged_kernel_sources():
+    import hashlib
     import bench
-    entry = dict(bench.TC2_TRAFFIC)
-    assert bench.profiled_traffic(entry) == entry["bytes"]
-    stale = dict(entry, sources_sha256="0" * 64)
+    root = os.path.dirname(os.path.abspath(bench.__file__))
+    h = hashlib.sha256()
+    for f in bench.TC2_TRAFFIC["sources"]:
+        with open(os.path.join(root, f), "rb") as fh:
+            h.update(fh.read())
+    current = dict(bench.TC2_TRAFFIC, sources_sha256=h.hexdigest())
+    assert bench.profiled_traffic(current) == current["bytes"]
+    stale = dict(current, sources_sha256="0" * 64)
     assert bench.profiled_traffic(stale) is None
-    missing = dict(entry, sources=["no/such/file.cu"])
+    missing = dict(current, sources=["no/such/file.cu"])
     assert bench.profiled_traffic(missing) is None
