@@ -330,8 +330,8 @@ w8a8_status int8_outlier_split(const void *X, int64_t M, int64_t K, int64_t ldx,
   DeviceInfo *d;
   if (w8a8_status s = device_info(&d)) return s;
   return from_cuda(launch_outlier_split(static_cast<const uint16_t *>(X), M, K, ldx, threshold, cap, Xq, S_x,
-                                        outlier_idx, n_out, static_cast<uint16_t *>(Xo), workspace, d->status,
-                                        static_cast<cudaStream_t>(stream)));
+                                        outlier_idx, n_out, static_cast<uint16_t *>(Xo), workspace, d->sm_count,
+                                        d->status, static_cast<cudaStream_t>(stream)));
 }
 
 w8a8_status int8_mixed_decomp_gemm(const int8_t *Xq, const float *S_x, const void *Xo,

@@ -74,7 +74,7 @@ int decode_split(int64_t M, int64_t N, int64_t K, bool fused_quant);
 // masked per-row quantization and outlier gather.
 cudaError_t launch_outlier_split(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, float threshold, int32_t cap,
                                  int8_t *Xq, float *S_x, int32_t *idx, int32_t *n_out, uint16_t *Xo, void *workspace,
-                                 int32_t *status, cudaStream_t s);
+                                 int num_sms, int32_t *status, cudaStream_t s);
 size_t outlier_workspace_bytes(int64_t K);
 
 // Per-device set-up of the C ABI (done once per device): SM count and the

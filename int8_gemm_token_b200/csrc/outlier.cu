@@ -29,9 +29,20 @@ namespace {
 constexpr int kRowsPerThread = 32;  // pass 1: rows per thread band
 
 // ------------------------------------------------------------------ pass 1
+// 16-byte load that asks L2 to keep the line (evict-last policy): pass 2 reads
+// X again, and X (67 MB at 4096 x 8192 bf16) fits in the 126 MB L2.
+__device__ __forceinline__ uint4 ld_keep_l2(const uint4 *p, uint64_t policy) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(policy));
+  return v;
+}
+
 __global__ void __launch_bounds__(256) outlier_colflag_kernel(const uint16_t *__restrict__ X, int64_t M, int64_t K,
                                                               int64_t ldx, float threshold,
                                                               uint32_t *__restrict__ bitmap) {
+  pdl_launch_dependents();  // the row pass may start: it reads only X until this pass completes
   const int64_t groups = K >> 3;  // 8-column groups
   const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (g >= groups) return;
@@ -41,11 +52,13 @@ __global__ void __launch_bounds__(256) outlier_colflag_kernel(const uint16_t *__
   uint32_t mx0 = 0, mx1 = 0, mx2 = 0, mx3 = 0;
   const uint4 *p = reinterpret_cast<const uint4 *>(X + r0 * ldx) + g;
   const int64_t step = ldx >> 3;
+  uint64_t keep;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
   int64_t r = r0;
   for (; r + 8 <= r1; r += 8) {
     uint4 v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __ldcs(p + i * step);
+    for (int i = 0; i < 8; ++i) v[i] = ld_keep_l2(p + i * step, keep);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       mx0 = __vmaxu2(mx0, v[i].x & 0x7FFF7FFFu);
@@ -56,7 +69,7 @@ __global__ void __launch_bounds__(256) outlier_colflag_kernel(const uint16_t *__
     p += 8 * step;
   }
   for (; r < r1; ++r) {
-    const uint4 v = __ldcs(p);
+    const uint4 v = ld_keep_l2(p, keep);
     mx0 = __vmaxu2(mx0, v.x & 0x7FFF7FFFu);
     mx1 = __vmaxu2(mx1, v.y & 0x7FFF7FFFu);
     mx2 = __vmaxu2(mx2, v.z & 0x7FFF7FFFu);
@@ -118,7 +131,19 @@ __device__ int32_t build_outlier_list(const uint32_t *__restrict__ bitmap, int64
 }
 
 // G threads per row (32: one warp per row, 8 rows per block; 256: one row per
-// block), VPT 16-byte chunks per thread held in registers.
+// block), VPT 16-byte chunks per thread held in registers. Each block builds
+// the outlier list and copies the column bitmap into shared memory once, then
+// walks its row groups (blockIdx.x, + gridDim.x, ...) with the next group's
+// loads in flight while the current one is reduced and quantized.
+template <int G, int VPT>
+__device__ __forceinline__ void load_row_chunks(const uint16_t *xrow, int64_t chunks, int t, bool ok, uint4 (&v)[VPT]) {
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int64_t c = t + static_cast<int64_t>(j) * G;
+    v[j] = (ok && c < chunks) ? __ldcs(reinterpret_cast<const uint4 *>(xrow) + c) : make_uint4(0, 0, 0, 0);
+  }
+}
+
 template <int G, int VPT>
 __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__restrict__ X, int64_t M, int64_t K,
                                                           int64_t ldx, const uint32_t *__restrict__ bitmap,
@@ -127,13 +152,32 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
                                                           int32_t *__restrict__ n_out, uint16_t *__restrict__ Xo,
                                                           int32_t *status) {
   constexpr int R = 256 / G;
-  extern __shared__ int32_t s_dyn[];  // cap entries of the index list
+  extern __shared__ int32_t s_dyn[];  // cap entries of the index list, then the column bitmap
   __shared__ int32_t s_scan[9];
-  __shared__ uint32_t red[8];
+  __shared__ uint32_t red[2][8];
   const int tid = threadIdx.x;
+  const int g = tid / G, t = tid % G;
+  const int64_t chunks = K >> 3;
+  const int64_t groups = (M + R - 1) / R;
+  int64_t grp = blockIdx.x;
+
+  // Launched with programmatic dependent launch, this kernel may start while
+  // the column-flag pass still runs. X is final by then (that pass started
+  // after everything before it completed), so the first rows' loads go out
+  // at once; the bitmap is read, and anything written, only after the wait.
+  uint4 v[VPT];
+  {
+    const int64_t m = grp * R + g;
+    load_row_chunks<G, VPT>(X + m * ldx, chunks, t, m < M, v);
+  }
+  pdl_wait_prerequisite();
+
   const int64_t words = (K + 31) >> 5;
   const int32_t total = build_outlier_list(bitmap, words, cap, s_dyn, s_scan);
   const int32_t nuse = total < cap ? total : cap;
+  uint32_t *s_bits = reinterpret_cast<uint32_t *>(s_dyn + (cap > 0 ? cap : 1));
+  for (int64_t w = tid; w < words; w += blockDim.x) s_bits[w] = __ldcg(bitmap + w);
+  __syncthreads();
   if (blockIdx.x == 0) {
     for (int j = tid; j < nuse; j += blockDim.x) out_idx[j] = s_dyn[j];
     if (tid == 0) {
@@ -142,70 +186,94 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
     }
   }
 
-  const int g = tid / G, t = tid % G;
-  const int64_t m = static_cast<int64_t>(blockIdx.x) * R + g;
-  const bool row_ok = m < M;
-  const int64_t chunks = K >> 3;
-  const uint16_t *xrow = X + m * ldx;
-  uint4 v[VPT];
-  uint32_t amax = 0;
+  for (int it = 0; grp < groups; grp += gridDim.x, ++it) {
+    const int64_t m = grp * R + g;
+    const bool row_ok = m < M;
+    // next group's loads, in flight while this one is processed (when the
+    // two rows fit in registers)
+    constexpr bool kPrefetch = VPT <= 8;
+    const int64_t mn = (grp + gridDim.x) * R + g;
+    const bool next_ok = grp + gridDim.x < groups && mn < M;
+    uint4 nxt[kPrefetch ? VPT : 1];
+    if constexpr (kPrefetch) load_row_chunks<G, VPT>(X + mn * ldx, chunks, t, next_ok, nxt);
+    uint32_t amax = 0;
 #pragma unroll
-  for (int j = 0; j < VPT; ++j) {
-    const int64_t c = t + static_cast<int64_t>(j) * G;
-    v[j] = make_uint4(0, 0, 0, 0);
-    if (row_ok && c < chunks) {
-      v[j] = __ldcs(reinterpret_cast<const uint4 *>(xrow) + c);
-      // zero the outlier columns of this 8-column chunk
-      const uint32_t mask8 = (__ldg(bitmap + ((c * 8) >> 5)) >> ((c * 8) & 31)) & 0xFFu;
-      if (mask8) {
-        uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+    for (int j = 0; j < VPT; ++j) {
+      const int64_t c = t + static_cast<int64_t>(j) * G;
+      if (row_ok && c < chunks) {
+        // zero the outlier columns of this 8-column chunk
+        const uint32_t mask8 = (s_bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+        if (mask8) {
+          uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          if (mask8 & (1u << (2 * h))) w[h] &= 0xFFFF0000u;
-          if (mask8 & (2u << (2 * h))) w[h] &= 0x0000FFFFu;
+          for (int h = 0; h < 4; ++h) {
+            if (mask8 & (1u << (2 * h))) w[h] &= 0xFFFF0000u;
+            if (mask8 & (2u << (2 * h))) w[h] &= 0x0000FFFFu;
+          }
+          v[j] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        v[j] = make_uint4(w[0], w[1], w[2], w[3]);
+        amax = absmax2_u4(v[j], amax);
       }
-      amax = absmax2_u4(v[j], amax);
+    }
+    amax = max(amax & 0xFFFFu, amax >> 16);
+    amax = __reduce_max_sync(0xFFFFFFFFu, amax);
+    if (G > 32) {  // one row per block: combine the warps (double-buffered, one barrier per row)
+      if ((tid & 31) == 0) red[it & 1][tid >> 5] = amax;
+      __syncthreads();
+      amax = red[it & 1][0];
+#pragma unroll
+      for (int w = 1; w < G / 32; ++w) amax = max(amax, red[it & 1][w]);
+    }
+    if (row_ok) {
+      const float a = __uint_as_float(amax << 16);
+      const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+      if (t == 0) S_x[m] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+      int8_t *qrow = Xq + m * K;
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int64_t c = t + static_cast<int64_t>(j) * G;
+        if (c < chunks) reinterpret_cast<uint2 *>(qrow)[c] = quant8_sym_sat(v[j], r);
+      }
+      // gather this row's outlier values (the row is hot in L1/L2)
+      const uint16_t *xrow = X + m * ldx;
+      for (int j = t; j < nuse; j += G) Xo[m * cap + j] = __ldg(xrow + s_dyn[j]);
+    }
+    if constexpr (kPrefetch) {
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) v[j] = nxt[j];
+    } else {
+      load_row_chunks<G, VPT>(X + mn * ldx, chunks, t, next_ok, v);
     }
   }
-  amax = max(amax & 0xFFFFu, amax >> 16);
-  amax = __reduce_max_sync(0xFFFFFFFFu, amax);
-  if (G > 32) {
-    if ((tid & 31) == 0) red[tid >> 5] = amax;
-    __syncthreads();
-    amax = red[0];
-#pragma unroll
-    for (int w = 1; w < G / 32; ++w) amax = max(amax, red[w]);
-  }
-  if (!row_ok) return;
-  const float a = __uint_as_float(amax << 16);
-  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
-  if (t == 0) S_x[m] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
-  int8_t *qrow = Xq + m * K;
-#pragma unroll
-  for (int j = 0; j < VPT; ++j) {
-    const int64_t c = t + static_cast<int64_t>(j) * G;
-    if (c < chunks) reinterpret_cast<uint2 *>(qrow)[c] = quant8_sym_sat(v[j], r);
-  }
-  // gather this row's outlier values (the row is hot in L1/L2)
-  for (int j = t; j < nuse; j += G) Xo[m * cap + j] = __ldg(xrow + s_dyn[j]);
 }
 
 template <int G, int VPT>
 cudaError_t launch_rows_t(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *bitmap,
                           int32_t cap, int8_t *Xq, float *S_x, int32_t *idx, int32_t *n_out, uint16_t *Xo,
-                          int32_t *status, cudaStream_t s) {
+                          int32_t num_sms, int32_t *status, cudaStream_t s) {
   constexpr int R = 256 / G;
-  const size_t smem = static_cast<size_t>(cap > 0 ? cap : 1) * sizeof(int32_t);
+  const size_t smem = static_cast<size_t>((cap > 0 ? cap : 1) + (K + 31) / 32) * sizeof(int32_t);
   auto kern = outlier_row_kernel<G, VPT>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  const unsigned blocks = static_cast<unsigned>((M + R - 1) / R);
-  kern<<<blocks, 256, smem, s>>>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status);
-  return cudaGetLastError();
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t groups = (M + R - 1) / R;
+  const int64_t resident = static_cast<int64_t>(num_sms) * (per_sm > 0 ? per_sm : 1);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(groups < resident ? groups : resident));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status);
 }
 
 }  // namespace
@@ -214,7 +282,7 @@ size_t outlier_workspace_bytes(int64_t K) { return static_cast<size_t>(((K + 31)
 
 cudaError_t launch_outlier_split(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, float threshold, int32_t cap,
                                  int8_t *Xq, float *S_x, int32_t *idx, int32_t *n_out, uint16_t *Xo, void *workspace,
-                                 int32_t *status, cudaStream_t s) {
+                                 int num_sms, int32_t *status, cudaStream_t s) {
   uint32_t *bitmap = static_cast<uint32_t *>(workspace);
   cudaError_t e = cudaMemsetAsync(bitmap, 0, outlier_workspace_bytes(K), s);
   if (e != cudaSuccess) return e;
@@ -224,13 +292,13 @@ cudaError_t launch_outlier_split(const uint16_t *X, int64_t M, int64_t K, int64_
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t chunks = K / 8;
-  if (chunks <= 32 * 4) return launch_rows_t<32, 4>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
-  if (chunks <= 32 * 8) return launch_rows_t<32, 8>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
-  if (chunks <= 32 * 16) return launch_rows_t<32, 16>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
-  if (chunks <= 256 * 4) return launch_rows_t<256, 4>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
-  if (chunks <= 256 * 8) return launch_rows_t<256, 8>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
-  if (chunks <= 256 * 16) return launch_rows_t<256, 16>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
-  return launch_rows_t<256, 32>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, status, s);
+  if (chunks <= 32 * 4) return launch_rows_t<32, 4>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, num_sms, status, s);
+  if (chunks <= 32 * 8) return launch_rows_t<32, 8>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, num_sms, status, s);
+  if (chunks <= 32 * 16) return launch_rows_t<32, 16>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, num_sms, status, s);
+  if (chunks <= 256 * 4) return launch_rows_t<256, 4>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, num_sms, status, s);
+  if (chunks <= 256 * 8) return launch_rows_t<256, 8>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, num_sms, status, s);
+  if (chunks <= 256 * 16) return launch_rows_t<256, 16>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, num_sms, status, s);
+  return launch_rows_t<256, 32>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, num_sms, status, s);
 }
 
 }  // namespace w8a8

@@ -47,7 +47,8 @@ def check_split(X, threshold, cap, ld_pad=0):
 
 @pytest.mark.parametrize("M,K,cols,ld_pad", [
     (3, 16, [2, 9], 0), (16, 256, [7, 100, 255], 8), (300, 4112, [0, 33, 4095, 4111], 0),
-    (129, 1024, [], 0), (2, 65536, [5, 65535], 0), (4096, 8192, [11, 512, 777, 4000, 6001, 8191], 0)])
+    (129, 1024, [], 0), (2, 65536, [5, 65535], 0), (4096, 8192, [11, 512, 777, 4000, 6001, 8191], 0),
+    (7, 24576, [100, 24575], 0), (1500, 16384, [3, 9000], 16), (20000, 512, [0, 511], 0)])
 def test_outlier_split_bit_exact(M, K, cols, ld_pad):
     X = planted(M, K, cols, seed=M + K)
     n, st = check_split(X, 6.0, 64, ld_pad)
