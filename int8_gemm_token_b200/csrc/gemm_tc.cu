@@ -171,6 +171,110 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&acc)[32], int64_
   }
 }
 
+// The same fixed-order epilogue for 32 columns, with the per-column constants
+// already in shared memory (s_sw = s_w[n]; s_add = 0 + bias[n] without the
+// side path, bias[n] with it; s_cs = colsum[n]; zeros past N).
+template <bool MIXED>
+__device__ __forceinline__ void epilogue_chunk_s(const uint32_t (&acc)[32], int64_t m, int64_t n0, int64_t M,
+                                                 int64_t N, float sx, int32_t z, const EpilogueArgs &ep,
+                                                 int32_t nuse, const float *s_sw, const float *s_add,
+                                                 const int32_t *s_cs) {
+  if (m >= M) return;
+  const bool full = n0 + 32 <= N;
+  float side[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) side[i] = 0.0f;
+  if (MIXED) {
+    for (int32_t j = 0; j < nuse; ++j) {
+      const float xo = __uint_as_float(static_cast<uint32_t>(ep.Xo[m * ep.cap + j]) << 16);
+      const uint16_t *wrow = ep.W + static_cast<int64_t>(__ldg(ep.outlier_idx + j)) * ep.ldw + n0;
+      if (full && (ep.ldw % 8) == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4 *>(wrow) + i);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            side[8 * i + 2 * h] = __fmaf_rn(xo, bf16_lo(w4[h]), side[8 * i + 2 * h]);
+            side[8 * i + 2 * h + 1] = __fmaf_rn(xo, bf16_hi(w4[h]), side[8 * i + 2 * h + 1]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (n0 + i < N) {
+            const float wv = __uint_as_float(static_cast<uint32_t>(__ldg(wrow + i)) << 16);
+            side[i] = __fmaf_rn(xo, wv, side[i]);
+          }
+        }
+      }
+    }
+  }
+  float y[32];
+  int32_t craw[32];
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    const float4 w = *reinterpret_cast<const float4 *>(s_sw + i);
+    const float4 a = *reinterpret_cast<const float4 *>(s_add + i);
+    const float sw4[4] = {w.x, w.y, w.z, w.w}, ad4[4] = {a.x, a.y, a.z, a.w};
+    int4 cs = make_int4(0, 0, 0, 0);
+    if (z != 0) cs = *reinterpret_cast<const int4 *>(s_cs + i);
+    const int32_t cs4[4] = {cs.x, cs.y, cs.z, cs.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      int32_t c = static_cast<int32_t>(acc[i + h]);
+      if (z != 0) c -= z * cs4[h];
+      craw[i + h] = c;
+      float add = ad4[h];
+      if (MIXED) add = ep.bias ? __fadd_rn(side[i + h], add) : side[i + h];
+      y[i + h] = __fmaf_rn(__int2float_rn(c), __fmul_rn(sx, sw4[h]), add);
+    }
+  }
+  if (ep.out_dtype == W8A8_BF16) {
+    uint16_t *o = static_cast<uint16_t *>(ep.out) + m * N + n0;
+    if (full && (N % 8) == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 v;
+        v.x = pack_bf16x2(y[8 * i + 0], y[8 * i + 1]);
+        v.y = pack_bf16x2(y[8 * i + 2], y[8 * i + 3]);
+        v.z = pack_bf16x2(y[8 * i + 4], y[8 * i + 5]);
+        v.w = pack_bf16x2(y[8 * i + 6], y[8 * i + 7]);
+        reinterpret_cast<uint4 *>(o)[i] = v;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (n0 + i < N) {
+          __nv_bfloat16 b = __float2bfloat16_rn(y[i]);
+          o[i] = *reinterpret_cast<uint16_t *>(&b);
+        }
+    }
+  } else if (ep.out_dtype == W8A8_FP32) {
+    float *o = static_cast<float *>(ep.out) + m * N + n0;
+    if (full && (N % 4) == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<float4 *>(o)[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (n0 + i < N) o[i] = y[i];
+    }
+  } else {
+    int32_t *o = static_cast<int32_t *>(ep.out) + m * N + n0;
+    if (full && (N % 4) == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<int4 *>(o)[i] = make_int4(craw[4 * i], craw[4 * i + 1], craw[4 * i + 2], craw[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (n0 + i < N) o[i] = craw[i];
+    }
+  }
+}
+
 template <int BN, int STAGES, bool MIXED>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -402,11 +506,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = base;
   uint8_t *sB = base + STAGES * kStageA2;
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sB + STAGES * kStageB2);
+  // per-column epilogue constants of the tile, one slot per accumulator:
+  // [slot][s_w | add | colsum][kTileN]
+  float *sConst = reinterpret_cast<float *>(sB + STAGES * kStageB2);
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sConst + 2 * 3 * kTileN);
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *tfull_bar = empty_bar + STAGES;
   uint64_t *tempty_bar = tfull_bar + 2;
-  uint64_t *drain_bar = tempty_bar + 2;
+  uint64_t *cready_bar = tempty_bar + 2;  // a slot of sConst is written (one arrival per epilogue warp)
+  uint64_t *drain_bar = cready_bar + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -425,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], 8);  // one arrival per epilogue warp of both CTAs
+      mbar_init(&cready_bar[b], 4);  // one arrival per epilogue warp of this CTA
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -548,6 +657,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kEpiWarp0) {
     pdl_wait_prerequisite();  // S_x, scales, side inputs and `out` belong to the previous kernel until then
     // -------------------------------------------------- epilogue (both CTAs)
+    // Per tile: the 4 epilogue warps stage the tile's per-column constants in
+    // shared memory while its MMAs run (64 columns each), then each warp turns
+    // its 32 accumulator rows into outputs, 32 columns at a time, with the
+    // next chunk's tcgen05.ld in flight while the current one is stored.
     const int q = warp - kEpiWarp0;
     const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
     int32_t nuse = 0;
@@ -555,7 +668,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t tile = cluster_id; tile < num_tiles; tile += num_clusters) {
-      const bool ready = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag, limit_ns));
+      if (*abort_flag) break;
+      const int64_t nbase = (tile / num_m) * kTileN;
+      float *c_sw = sConst + acc * 3 * kTileN, *c_add = c_sw + kTileN;
+      int32_t *c_cs = reinterpret_cast<int32_t *>(c_add + kTileN);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int col = q * 64 + j * 32 + lane;
+        const int64_t n = nbase + col;
+        float sw = 0.0f, add = 0.0f;
+        int32_t cs = 0;
+        if (n < N) {
+          sw = __ldg(ep.s_w + n);
+          if (ep.bias) add = MIXED ? __ldg(ep.bias + n) : __fadd_rn(0.0f, __ldg(ep.bias + n));
+          if (z != 0) cs = __ldg(ep.colsum + n);
+        }
+        c_sw[col] = sw;
+        c_add[col] = add;
+        c_cs[col] = cs;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cready_bar[acc]);
+      const bool ready =
+          __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&cready_bar[acc], acc_phase, abort_flag, limit_ns) &&
+                                      mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag, limit_ns));
       if (!ready) {
         if (lane == 0) {
           record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
@@ -565,16 +701,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int64_t m = (tile % num_m) * kTileM + rank * kHalf + q * 32 + lane;
-      const int64_t nbase = (tile / num_m) * kTileN;
       float sx = 0.0f;
       if (m < M) sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : __ldg(ep.S_x);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kTileN);
-#pragma unroll 1
-      for (int c = 0; c < kTileN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, r);
-        tmem_ld_wait();
-        epilogue_chunk<MIXED>(r, m, nbase + c * 32, M, N, sx, z, ep, nuse);
+      uint32_t ra[32], rb[32];
+      tmem_ld_32x32b_x32(taddr, ra);
+#pragma unroll
+      for (int c = 0; c < kTileN / 32; c += 2) {
+        tmem_ld_wait();  // chunk c in ra
+        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, rb);
+        epilogue_chunk_s<MIXED>(ra, m, nbase + c * 32, M, N, sx, z, ep, nuse, c_sw + c * 32, c_add + c * 32,
+                                c_cs + c * 32);
+        tmem_ld_wait();  // chunk c + 1 in rb
+        if (c + 2 < kTileN / 32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, ra);
+        epilogue_chunk_s<MIXED>(rb, m, nbase + (c + 1) * 32, M, N, sx, z, ep, nuse, c_sw + (c + 1) * 32,
+                                c_add + (c + 1) * 32, c_cs + (c + 1) * 32);
       }
       tc_fence_before();
       __syncwarp();
@@ -604,7 +745,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int STAGES, bool MIXED>
 cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                          const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
-  constexpr size_t kSmem = static_cast<size_t>(STAGES) * 2 * 128 * kBK + 1024 + 256;
+  constexpr size_t kSmem = static_cast<size_t>(STAGES) * 2 * 128 * kBK + 2 * 3 * 256 * 4 + 1024 + 256;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   alignas(64) CUtensorMap tmA, tmB;
   if (!encode_tmap_2d(&tmA, Xq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                       static_cast<uint64_t>(K), kBK, 128, true))
@@ -669,13 +811,12 @@ cudaError_t launch_tc_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N
 cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                            const EpilogueArgs &ep, bool mixed, int num_sms, int32_t *status,
                            cudaStream_t s) {
-  // CTA pairs (256-row tiles) once there are enough rows to fill them
-  // 7 stages of 32 KiB: the loaded L2/TMA latency is ~3000 cycles, and one
-  // stage is always being read by the MMAs, so six in flight keep the tensor
-  // pipe fed at 64 B/clk per SM.
+  // CTA pairs (256-row tiles) once there are enough rows to fill them.
+  // 6 stages of 32 KiB (a seventh measured no faster) leave room for the
+  // epilogue's per-column constants.
   if (M >= 256 && num_sms >= 2) {
-    if (mixed) return launch_tc2_t<7, true>(Xq, Wq, M, N, K, ep, num_sms, status, s);
-    return launch_tc2_t<7, false>(Xq, Wq, M, N, K, ep, num_sms, status, s);
+    if (mixed) return launch_tc2_t<6, true>(Xq, Wq, M, N, K, ep, num_sms, status, s);
+    return launch_tc2_t<6, false>(Xq, Wq, M, N, K, ep, num_sms, status, s);
   }
   if (mixed) return launch_tc_t<256, 4, true>(Xq, Wq, M, N, K, ep, num_sms, status, s);
   return launch_tc_t<256, 4, false>(Xq, Wq, M, N, K, ep, num_sms, status, s);
