@@ -704,18 +704,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sx = 0.0f;
       if (m < M) sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : __ldg(ep.S_x);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kTileN);
-      uint32_t ra[32], rb[32];
-      tmem_ld_32x32b_x32(taddr, ra);
+      if constexpr (MIXED) {
+        // the side path's epilogue is long: one chunk at a time, constants
+        // read per chunk (measured faster here than the staged form)
+#pragma unroll 1
+        for (int c = 0; c < kTileN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, r);
+          tmem_ld_wait();
+          epilogue_chunk<MIXED>(r, m, nbase + c * 32, M, N, sx, z, ep, nuse);
+        }
+      } else {
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32(taddr, ra);
 #pragma unroll
-      for (int c = 0; c < kTileN / 32; c += 2) {
-        tmem_ld_wait();  // chunk c in ra
-        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, rb);
-        epilogue_chunk_s<MIXED>(ra, m, nbase + c * 32, M, N, sx, z, ep, nuse, c_sw + c * 32, c_add + c * 32,
-                                c_cs + c * 32);
-        tmem_ld_wait();  // chunk c + 1 in rb
-        if (c + 2 < kTileN / 32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, ra);
-        epilogue_chunk_s<MIXED>(rb, m, nbase + (c + 1) * 32, M, N, sx, z, ep, nuse, c_sw + (c + 1) * 32,
-                                c_add + (c + 1) * 32, c_cs + (c + 1) * 32);
+        for (int c = 0; c < kTileN / 32; c += 2) {
+          tmem_ld_wait();  // chunk c in ra
+          tmem_ld_32x32b_x32(taddr + (c + 1) * 32, rb);
+          epilogue_chunk_s<MIXED>(ra, m, nbase + c * 32, M, N, sx, z, ep, nuse, c_sw + c * 32, c_add + c * 32,
+                                  c_cs + c * 32);
+          tmem_ld_wait();  // chunk c + 1 in rb
+          if (c + 2 < kTileN / 32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, ra);
+          epilogue_chunk_s<MIXED>(rb, m, nbase + (c + 1) * 32, M, N, sx, z, ep, nuse, c_sw + (c + 1) * 32,
+                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32);
+        }
       }
       tc_fence_before();
       __syncwarp();
