@@ -45,10 +45,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_count(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
                "r"(bytes)
@@ -206,11 +202,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Named barrier among `count` threads (id 1..15; id 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialization may start while the previous kernel in the stream is still
 // running; griddepcontrol.wait blocks until that kernel has completed and its
@@ -224,17 +215,6 @@ __device__ __forceinline__ void pdl_wait_prerequisite() {
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
-
-// atomicAdd with release semantics at GPU scope: every write that precedes it
-// (including other threads' writes ordered before it by a barrier) is visible
-// before the addition is.
-__device__ __forceinline__ uint32_t atomic_add_release_gpu(uint32_t *p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
-__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 // ---------------------------------------------------------------- CTA pairs
 // Rank of this CTA in its cluster.
@@ -330,12 +310,6 @@ __device__ __forceinline__ int rne_clamped(float p) {
 __device__ __forceinline__ int rne_s32(float p) {
   int r;
   asm("cvt.rni.s32.f32 %0, %1;" : "=r"(r) : "f"(p));
-  return r;
-}
-
-__device__ __forceinline__ int add_sat_s32(int a, int b) {
-  int r;
-  asm("add.sat.s32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 
