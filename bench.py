@@ -168,6 +168,12 @@ def whole_job_tops(ops_per_rank_step: float, world: int, ms_per_step: float) -> 
     return world * ops_per_rank_step / (ms_per_step * 1e-3) / 1e12
 
 
+def workload_config(world: int) -> dict:
+    """The `config` of the JSON line; both arms report the same one."""
+    return {"workload": WORKLOAD, "M": M, "K": K, "N": N, "parallelism": f"replicas x{world}",
+            "l2": f"{N_SETS} rotating X/Wq/out sets, {N_SETS * 115} MB > 126 MB L2"}
+
+
 def cpu_baseline_sample(rows: int, seed: int = 0):
     """Time the oracle on `rows` tokens of the workload: per-token quant,
     int64 GEMM and the fixed-order epilogue. Returns (seconds, ops)."""
@@ -202,7 +208,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N},
+            "data": "synthetic", "config": workload_config(world),
             "cpu_baseline": {"value": value, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -346,8 +352,7 @@ def run_ours(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "parallelism": f"replicas x{world}",
-                       "l2": f"{N_SETS} rotating X/Wq/out sets, {N_SETS * 115} MB > 126 MB L2"},
+            "config": workload_config(world),
             "roofline": {"bound": "tensor", "kernel": "gemm_i8_tc2_kernel", "achieved": gemm_tops,
                          "peak": int8_sustained, "unit": "TOPS", "frac": gemm_tops / int8_sustained,
                          "peak_source": f"{peaks['source']} sustained bf16 {peaks['bf16_tflops_sustained']} TFLOP/s x 2 "
