@@ -66,7 +66,7 @@ TC2_TRAFFIC = {
     "bytes": 53_721_088 + 6_855_936,
     "sources": ["int8_gemm_token_b200/csrc/gemm_tc.cu", "int8_gemm_token_b200/csrc/device.cuh",
                 "int8_gemm_token_b200/csrc/kernels.h"],
-    "sources_sha256": "8269064042a6fbcb5a12ad87d6e497f7555002c7104828a682f8fc36c846b86a",
+    "sources_sha256": "cac78c3fc48a2e57b101eab9ea5270dad2fa659ce0577abf32eaaf8089c79a60",
     "profile": "profiles/gemm_i8_tc2_prefill_7b_2048x4096x11008.txt",
 }
 

@@ -505,11 +505,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // without it the driver may size the carveout for one CTA per SM.
 template <int MP, int SPLIT, bool FUSEQ>
 cudaError_t configure_decode_kernel() {
-  auto kern = gemm_i8_decode_kernel<MP, SPLIT, FUSEQ>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(DecCfg<MP, SPLIT, FUSEQ>::kSmem));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  return ensure_kernel_smem<gemm_i8_decode_kernel<MP, SPLIT, FUSEQ>>(static_cast<int>(DecCfg<MP, SPLIT, FUSEQ>::kSmem),
+                                                                     true);
 }
 
 // The activation operand: int8 Xq [M, K] (row stride ldx bytes) or, with

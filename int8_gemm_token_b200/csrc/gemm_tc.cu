@@ -767,7 +767,7 @@ cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t 
                       static_cast<uint64_t>(K), kBK, 128, true))
     return cudaErrorInvalidValue;
   auto kern = gemm_i8_tc2_kernel<STAGES, MIXED>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+  cudaError_t e = ensure_kernel_smem<gemm_i8_tc2_kernel<STAGES, MIXED>>(static_cast<int>(kSmem), false);
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
   const int64_t pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
@@ -801,8 +801,7 @@ cudaError_t launch_tc_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N
     return cudaErrorInvalidValue;
   auto kern = gemm_i8_tc_kernel<BN, STAGES, MIXED>;
   // per function and per device; cheap enough to repeat on every launch
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(Cfg::kSmem));
+  cudaError_t e = ensure_kernel_smem<gemm_i8_tc_kernel<BN, STAGES, MIXED>>(static_cast<int>(Cfg::kSmem), false);
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
   cudaLaunchConfig_t cfg = {};

@@ -2,6 +2,8 @@
 // include/w8a8.h). Every launcher returns the launch's cudaError_t.
 #pragma once
 
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -29,6 +31,28 @@ struct EpilogueArgs {
   void *out = nullptr;  // [M, N] dense
   int32_t out_dtype = W8A8_BF16;
 };
+
+// Once per kernel and device: raise the kernel's dynamic shared-memory limit to
+// at least `bytes` (and ask for the largest shared-memory carveout). Later
+// calls with no larger size skip the driver calls.
+template <auto Kernel>
+cudaError_t ensure_kernel_smem(int bytes, bool max_carveout) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> set_bytes[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && set_bytes[dev].load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && max_carveout)
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
+    int prev = set_bytes[dev].load(std::memory_order_relaxed);
+    while (prev < bytes && !set_bytes[dev].compare_exchange_weak(prev, bytes)) {
+    }
+  }
+  return e;
+}
 
 cudaError_t launch_quant_per_token(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                    int8_t *Xq, float *S_x, cudaStream_t s);

@@ -255,7 +255,7 @@ cudaError_t launch_rows_t(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, 
   const size_t smem = static_cast<size_t>((cap > 0 ? cap : 1) + (K + 31) / 32) * sizeof(int32_t);
   auto kern = outlier_row_kernel<G, VPT>;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = ensure_kernel_smem<outlier_row_kernel<G, VPT>>(static_cast<int>(smem), false);
     if (e != cudaSuccess) return e;
   }
   int per_sm = 0;
