@@ -66,7 +66,7 @@ TC2_TRAFFIC = {
     "bytes": 53_721_088 + 6_855_936,
     "sources": ["int8_gemm_token_b200/csrc/gemm_tc.cu", "int8_gemm_token_b200/csrc/device.cuh",
                 "int8_gemm_token_b200/csrc/kernels.h"],
-    "sources_sha256": "cac78c3fc48a2e57b101eab9ea5270dad2fa659ce0577abf32eaaf8089c79a60",
+    "sources_sha256": "6e4f8a76d59bc909485c44414113c931bc57326bf432664a0e469d729b47a0c8",
     "profile": "profiles/gemm_i8_tc2_prefill_7b_2048x4096x11008.txt",
 }
 

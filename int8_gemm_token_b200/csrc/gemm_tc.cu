@@ -38,7 +38,9 @@ struct TcConfig {
   static constexpr int kStageB = BN * kBK;
   static constexpr int kTmemCols = 2 * BN;  // two accumulators
   static constexpr size_t kRing = static_cast<size_t>(STAGES) * (kStageA + kStageB);
-  static constexpr size_t kSmem = kRing + 1024 /*alignment slack*/ + 256 /*barriers etc.*/;
+  static constexpr size_t kSmem = kRing + 2 * 3 * BN * 4 /*epilogue constants*/ + 1024 /*alignment slack*/ +
+                                  256 /*barriers etc.*/;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
 };
 
@@ -286,11 +288,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = base;
   uint8_t *sB = base + STAGES * kStageA;
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(base + Cfg::kRing);
+  // per-column epilogue constants of the tile, one slot per accumulator:
+  // [slot][s_w | add | colsum][BN]
+  float *sConst = reinterpret_cast<float *>(base + Cfg::kRing);
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sConst + 2 * 3 * BN);
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *tfull_bar = empty_bar + STAGES;
   uint64_t *tempty_bar = tfull_bar + 2;
-  uint64_t *drain_bar = tempty_bar + 2;
+  uint64_t *cready_bar = tempty_bar + 2;  // a slot of sConst is written (one arrival per epilogue warp)
+  uint64_t *drain_bar = cready_bar + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -307,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], 4);  // one arrival per epilogue warp
+      mbar_init(&cready_bar[b], 4);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -431,6 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kEpiWarp0) {
     pdl_wait_prerequisite();  // S_x, scales, side inputs and `out` belong to the previous kernel until then
     // -------------------------------------------------- epilogue
+    // As in the CTA-pair kernel: the tile's per-column constants are staged in
+    // shared memory while its MMAs run, and (without the side path) the next
+    // chunk's tcgen05.ld is in flight while the current one is stored.
     const int q = warp - kEpiWarp0;  // TMEM lane quarter of this warp (warp % 4)
     const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
     int32_t nuse = 0;
@@ -438,8 +448,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      // tcgen05.ld is warp-collective: the whole warp goes on or gives up together
-      const bool ready = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag, limit_ns));
+      if (*abort_flag) break;
+      const int64_t nbase = (tile / num_m) * BN;
+      float *c_sw = sConst + acc * 3 * BN, *c_add = c_sw + BN;
+      int32_t *c_cs = reinterpret_cast<int32_t *>(c_add + BN);
+      if constexpr (!MIXED) {
+#pragma unroll
+        for (int j = 0; j < BN / 128; ++j) {
+          const int col = q * (BN / 4) + j * 32 + lane;
+          const int64_t n = nbase + col;
+          float sw = 0.0f, add = 0.0f;
+          int32_t cs = 0;
+          if (n < N) {
+            sw = __ldg(ep.s_w + n);
+            if (ep.bias) add = __fadd_rn(0.0f, __ldg(ep.bias + n));
+            if (z != 0) cs = __ldg(ep.colsum + n);
+          }
+          c_sw[col] = sw;
+          c_add[col] = add;
+          c_cs[col] = cs;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cready_bar[acc]);
+      const bool ready =
+          __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&cready_bar[acc], acc_phase, abort_flag, limit_ns) &&
+                                      mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag, limit_ns));
       if (!ready) {
         if (lane == 0) {
           record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
@@ -449,16 +483,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int64_t m = (tile % num_m) * kBM + q * 32 + lane;
-      const int64_t nbase = (tile / num_m) * BN;
       float sx = 0.0f;
       if (m < M) sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : __ldg(ep.S_x);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      if constexpr (MIXED) {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, r);
-        tmem_ld_wait();
-        epilogue_chunk<MIXED>(r, m, nbase + c * 32, M, N, sx, z, ep, nuse);
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, r);
+          tmem_ld_wait();
+          epilogue_chunk<MIXED>(r, m, nbase + c * 32, M, N, sx, z, ep, nuse);
+        }
+      } else {
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32(taddr, ra);
+#pragma unroll
+        for (int c = 0; c < BN / 32; c += 2) {
+          tmem_ld_wait();  // chunk c in ra
+          tmem_ld_32x32b_x32(taddr + (c + 1) * 32, rb);
+          epilogue_chunk_s<MIXED>(ra, m, nbase + c * 32, M, N, sx, z, ep, nuse, c_sw + c * 32, c_add + c * 32,
+                                  c_cs + c * 32);
+          tmem_ld_wait();  // chunk c + 1 in rb
+          if (c + 2 < BN / 32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, ra);
+          epilogue_chunk_s<MIXED>(rb, m, nbase + (c + 1) * 32, M, N, sx, z, ep, nuse, c_sw + (c + 1) * 32,
+                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -673,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float *c_sw = sConst + acc * 3 * kTileN, *c_add = c_sw + kTileN;
       int32_t *c_cs = reinterpret_cast<int32_t *>(c_add + kTileN);
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      for (int j = 0; j < (MIXED ? 0 : 2); ++j) {
         const int col = q * 64 + j * 32 + lane;
         const int64_t n = nbase + col;
         float sw = 0.0f, add = 0.0f;
