@@ -103,8 +103,10 @@ def _rand_case(M, N, K, seed):
     return X, Wf, b
 
 
+# 32 < M < 256 takes the 1-CTA kernel (128 x 256 tiles), with ragged edges.
 @pytest.mark.parametrize("M,N,K", [(16, 512, 256), (128, 256, 128), (300, 520, 400), (1, 40, 16),
-                                   (257, 1000, 4096), (129, 257, 144), (520, 5400, 400), (520, 5000, 144)])
+                                   (257, 1000, 4096), (129, 257, 144), (520, 5400, 400), (520, 5000, 144),
+                                   (200, 11008, 256), (100, 2000, 400), (250, 40000, 128)])
 def test_gemm_int32_accumulator_bit_exact(M, N, K):
     X, Wf, b = _rand_case(M, N, K, M + N + K)
     rq, rS = oracle.quant_per_token(X)
@@ -116,7 +118,7 @@ def test_gemm_int32_accumulator_bit_exact(M, N, K):
 # M >= 256 takes the CTA-pair kernel: ragged last row and column tiles, K not a
 # multiple of the 128-byte k-block.
 @pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 400), (200, 264, 512), (520, 5000, 400),
-                                   (520, 5400, 256), (520, 5800, 272)])
+                                   (520, 5400, 256), (520, 5800, 272), (200, 11008, 512), (100, 2000, 400)])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_prefill_linear_bit_exact(M, N, K, out_dtype):
     X, Wf, b = _rand_case(M, N, K, 3 * M + N)
