@@ -149,7 +149,7 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
  *   out     device [M, N] dense, out_dtype W8A8_BF16, W8A8_FP32 or W8A8_I32
  *   workspace/workspace_bytes: accepted for compatibility with
  *           w8a8_linear_static and not used by this call (NULL/0 allowed).
- * M <= 32 (Decode-shaped) runs a weight-streaming kernel: one cluster of up to
+ * M <= 64 (Decode-shaped) runs a weight-streaming kernel: one cluster of up to
  * 8 CTAs per 128 output channels splits K, and the partial int32 sums are
  * added in distributed shared memory, so the call keeps no state in device
  * memory between calls and calls on different streams may overlap.
@@ -185,10 +185,11 @@ size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * shared memory before its MMAs read it, and no workspace is used (NULL
  * allowed). Other shapes quantize into the workspace with a separate kernel
  * first (every 128-channel tile of the fused kernel re-quantizes the whole
- * activation, which costs more than it saves there). The Decode-shaped
- * kernels use programmatic dependent launch like the Decode-shaped
- * w8a8_gemm_dequant (they stream their first weight tiles while the previous
- * kernel finishes); the rule on writing Wq given there applies.
+ * activation, which costs more than it saves there), then run the
+ * Decode-shaped GEMM for M <= 64 and the tile GEMM beyond. All of these
+ * kernels use programmatic dependent launch (they stream their first weight
+ * tiles while the previous kernel finishes); the rule on writing Wq given for
+ * w8a8_gemm_dequant applies.
  * Source: PDMIX glossary §2.2 (Decode has few tokens and is latency bound, so
  * a per-step quantization launch would be visible overhead) and §2.3 eq.
  * Q_decode; the hardware-acceleration chapter's note that decode is memory

@@ -198,8 +198,10 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
                                            d->sm_count, static_cast<cudaStream_t>(stream)));
 }
 
-// Decode-shaped calls (at most this many tokens) take the weight-streaming kernel.
-constexpr int64_t kDecodeMaxM = 32;
+// Calls with at most this many tokens take the weight-streaming decode kernel
+// (with the int8 activation); the one-kernel Decode linear serves up to 32.
+constexpr int64_t kDecodeMaxM = 64;
+constexpr int64_t kFusedMaxM = 32;
 
 static size_t align256(int64_t n) { return static_cast<size_t>(((n + 255) / 256) * 256); }
 
@@ -208,14 +210,14 @@ static size_t align256(int64_t n) { return static_cast<size_t>(((n + 255) / 256)
 // ALU operations per weight byte streamed: hidden behind the weight stream for
 // up to 16 tokens, and for N <= 4096 (few tiles, deep K split); beyond that
 // the separate quantization kernel (once per call) is faster on B200.
-static bool decode_fuses_quant(int64_t M, int64_t N) { return M <= 16 || N <= 4096; }
+static bool decode_fuses_quant(int64_t M, int64_t N) { return M <= 16 || (M <= kFusedMaxM && N <= 4096); }
 
 size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   // w8a8_linear_static keeps the statically quantized activation here unless
   // its Decode-shaped GEMM kernel quantizes it; the GEMM kernels themselves
   // need no workspace.
-  return M <= kDecodeMaxM && decode_fuses_quant(M, N) ? 0 : align256(M * K);
+  return decode_fuses_quant(M, N) ? 0 : align256(M * K);
 }
 
 static w8a8_status check_gemm_common(const int8_t *Xq, const int8_t *Wq, const float *s_w,
@@ -291,7 +293,7 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
   ep.bias = bias;
   ep.out = out;
   ep.out_dtype = out_dtype;
-  if (M <= kDecodeMaxM && decode_fuses_quant(M, N))  // one kernel: the GEMM quantizes each k-block
+  if (decode_fuses_quant(M, N))  // one kernel: the GEMM quantizes each k-block
     return from_cuda(launch_linear_static_decode(static_cast<const uint16_t *>(X), ldx, r, Z, Wq, M, N, K, ep,
                                                  d->status, st));
   if (M <= kDecodeMaxM) {

@@ -1,4 +1,4 @@
-// gemm_decode.cu -- Decode-shaped W8A8 linear (1..32 tokens): the GEMM is a
+// gemm_decode.cu -- Decode-shaped W8A8 linear (1..64 tokens): the GEMM is a
 // stream of the INT8 weight from HBM, so the kernel is organised around
 // keeping enough of that stream in flight on every SM that takes part.
 //
@@ -10,7 +10,7 @@
 //
 // How (sm_100a):
 //   * swap-AB: 128 rows of Wq [N, K] are the MMA's M dimension (TMEM lanes);
-//     the tokens, padded to MP = 16 or 32, are the MMA's N dimension;
+//     the tokens, padded to MP = 16, 32 or 64, are the MMA's N dimension;
 //   * one cluster of SPLIT CTAs per 128-row tile; CTA rank r of the cluster
 //     owns the k-blocks [r nkb / SPLIT, (r+1) nkb / SPLIT). SPLIT (1..8) is
 //     the largest that keeps tiles x SPLIT within one wave of two CTAs per SM,
@@ -85,7 +85,7 @@ struct DecCfg {
   static constexpr int kStagesFit = (kBudget - kRedBytes) / kStage;
   static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
   static constexpr size_t kSmem = static_cast<size_t>(kStages) * kStage + kRedBytes + 1024 + 256;
-  static constexpr int kTmemCols = 32;
+  static constexpr int kTmemCols = MP < 32 ? 32 : MP;  // one int32 column per padded token
   static_assert(kR % 8 == 0, "owned rows in 8-row groups");
   static_assert(kStageX % 1024 == 0 && kStageXb % 1024 == 0, "1 KiB alignment of activation stages");
   static_assert(kStages >= 3, "ring depth");
@@ -427,10 +427,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       tc_fence_after();
       uint32_t acc[MP];
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>((warp - kEpiWarp0) * 32) << 16);
-      if constexpr (MP == 32)
+      if constexpr (MP == 64) {
+        tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
+        tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
+      } else if constexpr (MP == 32) {
         tmem_ld_32x32b_x32(taddr, acc);
-      else
+      } else {
         tmem_ld_32x32b_x16(taddr, acc);
+      }
       tmem_ld_wait();
       tc_fence_before();
       if (owner == rank) {
@@ -644,14 +648,16 @@ cudaError_t launch_decode_mp(const DecodeActivation &act, const int8_t *Wq, int6
 
 int decode_split(int64_t M, int64_t N, int64_t K, bool fused_quant) {
   if (fused_quant) return M <= 16 ? decode_split_mp<16, true>(N, K) : decode_split_mp<32, true>(N, K);
-  return M <= 16 ? decode_split_mp<16, false>(N, K) : decode_split_mp<32, false>(N, K);
+  if (M <= 16) return decode_split_mp<16, false>(N, K);
+  return M <= 32 ? decode_split_mp<32, false>(N, K) : decode_split_mp<64, false>(N, K);
 }
 
 cudaError_t launch_gemm_decode(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                                const EpilogueArgs &ep, int32_t *status, cudaStream_t s) {
   const DecodeActivation act{Xq, ldx, nullptr, nullptr};
   if (M <= 16) return launch_decode_mp<16, false>(act, Wq, M, N, K, ep, status, s);
-  return launch_decode_mp<32, false>(act, Wq, M, N, K, ep, status, s);
+  if (M <= 32) return launch_decode_mp<32, false>(act, Wq, M, N, K, ep, status, s);
+  return launch_decode_mp<64, false>(act, Wq, M, N, K, ep, status, s);
 }
 
 cudaError_t launch_linear_static_decode(const uint16_t *X, int64_t ldx, const float *r, const int32_t *Z,

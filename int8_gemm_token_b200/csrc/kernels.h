@@ -75,7 +75,7 @@ cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_t s);
 
-// Decode-shaped GEMM (M <= 32): one cluster of decode_split(M, N, K) CTAs
+// Decode-shaped GEMM (M <= 64): one cluster of decode_split(M, N, K) CTAs
 // per 128-row weight tile, partial sums reduced through distributed shared
 // memory (no workspace). Launched with programmatic dependent launch: it may
 // start while the previous kernel in the stream runs, streams its first
@@ -84,9 +84,9 @@ cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_
 // dependents launch early must not write Wq).
 cudaError_t launch_gemm_decode(const int8_t *Xq, int64_t ldx, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                                const EpilogueArgs &ep, int32_t *status, cudaStream_t s);
-// The Decode linear in one kernel: the same GEMM, with the static per-tensor
-// quantization of bf16 X (row stride ldx elements, device scalars r and Z)
-// done inside it on each activation k-block before the MMAs read it.
+// The Decode linear in one kernel (M <= 32): the same GEMM, with the static
+// per-tensor quantization of bf16 X (row stride ldx elements, device scalars
+// r and Z) done inside it on each activation k-block before the MMAs read it.
 cudaError_t launch_linear_static_decode(const uint16_t *X, int64_t ldx, const float *r, const int32_t *Z,
                                         const int8_t *Wq, int64_t M, int64_t N, int64_t K, const EpilogueArgs &ep,
                                         int32_t *status, cudaStream_t s);

@@ -22,7 +22,7 @@ HEADER = os.path.join(ROOT, "include", "w8a8.h")
 
 OK = 0
 BF16, FP32, I32 = 0, 1, 2
-DECODE_MAX_M = 32  # calls with at most this many tokens take the weight-streaming decode kernel
+DECODE_MAX_M = 64  # calls with at most this many tokens take the weight-streaming decode kernel
 STATUS_NAMES = {}
 
 

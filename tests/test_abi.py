@@ -107,5 +107,6 @@ def test_valid_call_without_a_gpu_reports_no_device(L):
     assert w8a8.w8a8_gemm_workspace_size(4, 8, 64) == 0  # one kernel: quantized inside the GEMM
     assert w8a8.w8a8_gemm_workspace_size(32, 4096, 64) == 0
     assert w8a8.w8a8_gemm_workspace_size(32, 4104, 64) >= 32 * 64  # quantization kernel first
+    assert w8a8.w8a8_gemm_workspace_size(48, 100, 64) >= 48 * 64  # 33..64 tokens: quantization kernel first
     assert w8a8.w8a8_gemm_workspace_size(64, 8, 64) >= 64 * 64
     assert w8a8.lib().int8_outlier_split_workspace_size(8192) >= 8192 // 8

@@ -203,7 +203,8 @@ def test_bounded_wait_reports_timeout_and_device_stays_usable():
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (5, 300, 400), (16, 4096, 4096), (17, 520, 1024),
                                    (32, 11008, 4096), (3, 40, 16), (32, 4096, 11008), (32, 22016, 4096),
                                    (32, 131072, 512), (16, 131072, 256), (32, 1024, 4096), (8, 256, 2048),
-                                   (32, 5376, 4096), (16, 6272, 2048), (7, 7552, 1552), (32, 2816, 4096)])
+                                   (32, 5376, 4096), (16, 6272, 2048), (7, 7552, 1552), (32, 2816, 4096),
+                                   (33, 11008, 4096), (48, 4096, 1552), (64, 22016, 512), (64, 520, 4096)])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.int32])
 def test_decode_gemm_int8_input_bit_exact(M, N, K, out_dtype):
     """Small-M GEMM (K split over a cluster of 1..8 CTAs per 128 output
@@ -222,7 +223,8 @@ def test_decode_gemm_int8_input_bit_exact(M, N, K, out_dtype):
 
 @pytest.mark.parametrize("M,N,K,ld_pad", [(3, 200, 400, 8), (32, 384, 2048, 0), (9, 12288, 4096, 0),
                                           (32, 22016, 4096, 0), (32, 4096, 11008, 0), (32, 131072, 512, 0),
-                                          (12, 65536, 1024, 24), (32, 5376, 4096, 0), (7, 7552, 1552, 8)])
+                                          (12, 65536, 1024, 24), (32, 5376, 4096, 0), (7, 7552, 1552, 8),
+                                          (64, 11008, 4096, 0), (40, 300, 400, 8)])
 def test_decode_fused_static_ragged_and_block_shapes(M, N, K, ld_pad):
     case = synth.decode_static(M=M, N=N, K=K, seed=M + N)
     S, r, Z = W.w8a8_calibrate_static(dev_bf16(case.Xcal))
