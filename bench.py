@@ -66,7 +66,7 @@ TC2_TRAFFIC = {
     "bytes": 53_721_088 + 6_855_936,
     "sources": ["int8_gemm_token_b200/csrc/gemm_tc.cu", "int8_gemm_token_b200/csrc/device.cuh",
                 "int8_gemm_token_b200/csrc/kernels.h"],
-    "sources_sha256": "6e4f8a76d59bc909485c44414113c931bc57326bf432664a0e469d729b47a0c8",
+    "sources_sha256": "79e222cd70422b034c665e9bcedb377052c131ee43bd7ba6a03f5da159c55275",
     "profile": "profiles/gemm_i8_tc2_prefill_7b_2048x4096x11008.txt",
 }
 
