@@ -13,21 +13,29 @@
 //     the tokens, padded to MP = 16, 32 or 64, are the MMA's N dimension;
 //   * one cluster of SPLIT CTAs per 128-row tile; CTA rank r of the cluster
 //     owns the k-blocks [r nkb / SPLIT, (r+1) nkb / SPLIT). SPLIT (1..8) is
-//     the largest that keeps tiles x SPLIT within one wave of two CTAs per SM,
-//     so small N still spreads over the GPU and large N needs no split;
+//     the largest whose clusters are all resident at once (with at least two
+//     k-blocks per CTA), so small N still spreads over the GPU and large N
+//     needs no split;
 //   * CTAs are small (~100 KiB of shared memory) so that two share an SM:
 //     that doubles the copies in flight per SM and lets the next kernel's
 //     CTAs start streaming while this kernel's last CTAs finish;
-//   * warp 0 streams the weight tile and the matching int8 activation k-block
-//     through a TMA ring (5-6 x (16 KiB + MP x 128 B), 128B swizzle); warp 1
-//     issues tcgen05.mma kind::i8 (M = 128, N = MP) into one TMEM accumulator;
-//   * warps 4-7 fetch the per-channel constants while the weight streams,
-//     then read the accumulator (tcgen05.ld) into registers. With SPLIT = 1
-//     they store the outputs from there. Otherwise, after a cluster barrier
-//     (every ring is free), each CTA stores its partial sums into the shared
-//     memory of the CTA that finishes those rows (st.shared::cluster); after
-//     a second barrier each CTA adds the SPLIT partials of its rows (exact
-//     int32), runs the epilogue and stores. No global workspace, no atomics;
+//   * warp 0 streams the weight tile and the matching activation k-block
+//     through a TMA ring (3-6 stages of 16 KiB + the activation, 128B
+//     swizzle); warp 1 issues tcgen05.mma kind::i8 (M = 128, N = MP) into
+//     one TMEM accumulator;
+//   * FUSEQ (the one-kernel Decode linear): the activation arrives as bf16,
+//     two [MP][64] boxes per k-block, and the four epilogue warps -- idle
+//     until the last MMA -- quantize it into the 128B-swizzled int8 operand,
+//     fence it for the tensor core and signal a per-stage barrier that the
+//     MMA issuer also waits on;
+//   * when the accumulator is full, each epilogue thread holds one weight row
+//     for every token (tcgen05.ld). Rows are owned by cluster ranks in 8-row
+//     groups: a CTA keeps the partial sums of its own rows in its idle weight
+//     ring and stores the others into the owner's shared memory
+//     (st.shared::cluster). After one cluster barrier all 256 threads add the
+//     SPLIT partials (exact int32) of chunks of 8 outputs, run the epilogue
+//     with the per-channel constants fetched before the barrier, and store 16
+//     bytes at a time. No global workspace, no atomics;
 //   * programmatic dependent launch: the kernel lets its dependents launch
 //     as soon as it has started, and requests its first ring of weight tiles
 //     before it waits for the previous kernel in the stream
