@@ -66,7 +66,7 @@ TC2_TRAFFIC = {
     "bytes": 53_721_088 + 6_855_936,
     "sources": ["int8_gemm_token_b200/csrc/gemm_tc.cu", "int8_gemm_token_b200/csrc/device.cuh",
                 "int8_gemm_token_b200/csrc/kernels.h"],
-    "sources_sha256": "79e222cd70422b034c665e9bcedb377052c131ee43bd7ba6a03f5da159c55275",
+    "sources_sha256": "162deaec986b446b20d5d9bbdf721dbf707222c26f734c216e01986cf9b0fc16",
     "profile": "profiles/gemm_i8_tc2_prefill_7b_2048x4096x11008.txt",
 }
 
@@ -421,7 +421,7 @@ def bench_decode(args, dev, rank, peaks):
     def bf(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    rows = []
+    rows, requant = [], []
     for N in (11008, 4096):
         case = synth.decode_static(M=32, N=N, K=DEC_K, seed=rank)
         S, r, Z = W.w8a8_calibrate_static(bf(case.Xcal))
@@ -437,12 +437,31 @@ def bench_decode(args, dev, rank, peaks):
             nbytes = N * DEC_K + 8.0 * N + 2.0 * M * DEC_K + 2.0 * M * N
             gbs = nbytes / (us * 1e-6) / 1e9
             rows.append({"M": M, "K": DEC_K, "N": N, "us": us, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]})
+            # the int8 codes of the next linear straight from the epilogue, vs
+            # the bf16 output followed by the static quantization kernel (the
+            # next linear's r, Z stood in by this one's: same arithmetic)
+            q = torch.empty((M, N), dtype=torch.int8, device=dev)
+            rq_us = graph_time_us(lambda i: W.w8a8_linear_static_requant(X, S, r, Z, *ws[i % n_w], r, Z, out=q,
+                                                                         workspace=work), 2 * n_w)
+
+            def pair(i):
+                W.w8a8_linear_static(X, S, r, Z, *ws[i % n_w], out=out, workspace=work)
+                W.w8a8_quant_per_tensor(out, r, Z, Xq=q)
+            pair_us = graph_time_us(pair, 2 * n_w)
+            rq_bytes = N * DEC_K + 8.0 * N + 2.0 * M * DEC_K + 1.0 * M * N
+            rq_gbs = rq_bytes / (rq_us * 1e-6) / 1e9
+            requant.append({"M": M, "K": DEC_K, "N": N, "us": rq_us, "GB/s": rq_gbs, "frac": rq_gbs / peaks["hbm_gbs"],
+                            "unfused_us": pair_us})
         del ws
     # static quant alone vs GEMM alone (the C_s / C_g of the PDMIX cost model) at the largest shape
     return {"workload": "decode: static-quant W8A8 linear, w8a8_linear_static (one kernel with the quantization fused "
                         "into the weight-streaming GEMM for M <= 16 or N <= 4096, else quantization kernel + GEMM), "
                         "back-to-back calls, rotating weights > L2, CUDA-graph timed", "rows": rows,
-            "unit": "GB/s", "peak": peaks["hbm_gbs"], "algorithmic_bytes": "N*K + 8N + 2MK + 2MN per call"}
+            "unit": "GB/s", "peak": peaks["hbm_gbs"], "algorithmic_bytes": "N*K + 8N + 2MK + 2MN per call",
+            "requant": {"workload": "w8a8_linear_static_requant: the same Decode linear writing the next linear's "
+                                    "static int8 codes from its epilogue; unfused_us = w8a8_linear_static (bf16) + "
+                                    "w8a8_quant_per_tensor", "rows": requant,
+                        "algorithmic_bytes": "N*K + 8N + 2MK + MN per call"}}
 
 
 def bench_llm_int8(args, dev, rank, peaks, int8_peak):

@@ -207,6 +207,57 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
                                size_t workspace_bytes, void *stream);
 
 /*
+ * Decode linear whose result is handed to the next linear already quantized:
+ * w8a8_linear_static with a bf16 result, then that result quantized with the
+ * NEXT linear's static per-tensor parameters, in one call and with no bf16
+ * output written:
+ *   Xq_out[m, n] = clamp(rne(float(bf16(y[m, n])) * r_out) + Z_out, -128, 127)
+ * where y is the fp32 value of w8a8_linear_static's formula. The result is
+ * identical to w8a8_linear_static (out_dtype W8A8_BF16) followed by
+ * w8a8_quant_per_tensor(out, r_out, Z_out). The code is taken from the
+ * bf16-rounded value so that fusing changes no result.
+ * Source: PDMIX glossary §2.3 eq. Q_decode (the static scale and zero point
+ * of the next linear are known before the step runs) and §2.2 (Decode is
+ * latency bound, so the standalone quantization launch of each step is
+ * overhead); the hardware-acceleration chapter's note that runtimes fuse
+ * small operations into one kernel. No page fuses the two; this is a
+ * deployment entry point of this library.
+ *   X, S, r, Z, Wq, s_w, colsum, bias, workspace: as in w8a8_linear_static
+ *   r_out, Z_out  device scalars of the next linear (w8a8_calibrate_static)
+ *   Xq_out        device int8 [M, N] dense, 16-byte aligned, written
+ * M <= 64 only (the Decode-shaped kernels); larger M returns
+ * W8A8_ERR_UNSUPPORTED_SHAPE without launching anything. r_out and Z_out are
+ * read after the previous kernel on the stream has completed (the rule on
+ * writing Wq of w8a8_gemm_dequant applies).
+ */
+w8a8_status w8a8_linear_static_requant(const void *X, int64_t M, int64_t K, int64_t ldx, const float *S,
+                                       const float *r, const int32_t *Z, const int8_t *Wq,
+                                       const float *s_w, const int32_t *colsum, const float *bias,
+                                       int64_t N, const float *r_out, const int32_t *Z_out, int8_t *Xq_out,
+                                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * w8a8_gemm_dequant whose result is handed to the next linear already
+ * quantized: for int8 codes in (for example the output of
+ * w8a8_linear_static_requant), int8 codes of the next linear out, so that a
+ * chain of Decode linears passes no bf16 tensor between them.
+ *   Xq_out[m, n] = clamp(rne(float(bf16(y[m, n])) * r_out) + Z_out, -128, 127)
+ * with y the fp32 value of w8a8_gemm_dequant's formula: identical to
+ * w8a8_gemm_dequant (W8A8_BF16) followed by w8a8_quant_per_tensor(out,
+ * r_out, Z_out). Source and readings as for w8a8_linear_static_requant.
+ *   Xq, S_x, s_x_per_row, Z, Wq, s_w, colsum, bias: as in w8a8_gemm_dequant
+ *   r_out, Z_out  device scalars of the next linear
+ *   Xq_out        device int8 [M, N] dense, 16-byte aligned, written
+ * M <= 64 only (the Decode-shaped kernel); larger M returns
+ * W8A8_ERR_UNSUPPORTED_SHAPE. Programmatic dependent launch as in
+ * w8a8_gemm_dequant; r_out and Z_out are read after the previous kernel.
+ */
+w8a8_status w8a8_gemm_requant(const int8_t *Xq, const float *S_x, int32_t s_x_per_row, const int32_t *Z,
+                              const int8_t *Wq, const float *s_w, const int32_t *colsum, const float *bias,
+                              int64_t M, int64_t N, int64_t K, const float *r_out, const int32_t *Z_out,
+                              int8_t *Xq_out, void *stream);
+
+/*
  * w8a8_linear_static without a workspace argument: the same computation and
  * result as w8a8_linear_static (same arguments, same checks), for callers
  * that cannot allocate device memory when they run a Decode step -- a CUDA

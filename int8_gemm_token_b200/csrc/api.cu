@@ -264,6 +264,54 @@ w8a8_status w8a8_gemm_dequant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
                                   static_cast<cudaStream_t>(stream)));
 }
 
+w8a8_status w8a8_gemm_requant(const int8_t *Xq, const float *S_x, int32_t s_x_per_row, const int32_t *Z,
+                              const int8_t *Wq, const float *s_w, const int32_t *colsum, const float *bias,
+                              int64_t M, int64_t N, int64_t K, const float *r_out, const int32_t *Z_out,
+                              int8_t *Xq_out, void *stream) {
+  if (w8a8_status s = check_gemm_common(Xq, Wq, s_w, bias, colsum, M, N, K, Xq_out, W8A8_BF16)) return s;
+  if (M > kDecodeMaxM) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if (!S_x || (Z && !colsum) || !r_out || !Z_out) return W8A8_ERR_INVALID_ARG;
+  DeviceInfo *d;
+  if (w8a8_status s = device_info(&d)) return s;
+  EpilogueArgs ep;
+  ep.S_x = S_x;
+  ep.s_x_per_row = s_x_per_row ? 1 : 0;
+  ep.Z = Z;
+  ep.colsum = colsum;
+  ep.s_w = s_w;
+  ep.bias = bias;
+  ep.out = Xq_out;
+  ep.out_dtype = kOutRequantI8;
+  ep.r_out = r_out;
+  ep.z_out = Z_out;
+  return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, d->status, static_cast<cudaStream_t>(stream)));
+}
+
+// Shared by w8a8_linear_static and w8a8_linear_static_requant once their
+// arguments are checked: ep carries the epilogue operands and the output.
+static w8a8_status run_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx, const float *r,
+                                     const int32_t *Z, const int8_t *Wq, int64_t N, const EpilogueArgs &ep,
+                                     void *workspace, size_t workspace_bytes, cudaStream_t st) {
+  const size_t need = w8a8_gemm_workspace_size(M, N, K);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return W8A8_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return W8A8_ERR_MISALIGNED;
+  DeviceInfo *d;
+  if (w8a8_status s = device_info(&d)) return s;
+  if (decode_fuses_quant(M, N))  // one kernel: the GEMM quantizes each k-block
+    return from_cuda(launch_linear_static_decode(static_cast<const uint16_t *>(X), ldx, r, Z, Wq, M, N, K, ep,
+                                                 d->status, st));
+  // Static quantization into the workspace, then the GEMM; both use
+  // programmatic dependent launch, so the GEMM's weight stream starts while
+  // the quantization (and the previous kernel) run.
+  int8_t *Xq = static_cast<int8_t *>(workspace);
+  cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq, d->sm_count, st,
+                                          /*pdl=*/true);
+  if (e != cudaSuccess) return W8A8_ERR_CUDA;
+  if (M <= kDecodeMaxM) return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, d->status, st));
+  return from_cuda(launch_gemm_tc(Xq, Wq, M, N, K, ep, false, d->sm_count, d->status, st));
+}
+
 w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx, const float *S,
                                const float *r, const int32_t *Z, const int8_t *Wq,
                                const float *s_w, const int32_t *colsum, const float *bias,
@@ -278,12 +326,6 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
   if (!aligned16(Wq) || !aligned16(s_w) || !aligned16(colsum) || !aligned16(out) ||
       (bias && !aligned16(bias)))
     return W8A8_ERR_MISALIGNED;
-  const size_t need = w8a8_gemm_workspace_size(M, N, K);
-  if (need > 0 && (!workspace || workspace_bytes < need)) return W8A8_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return W8A8_ERR_MISALIGNED;
-  DeviceInfo *d;
-  if (w8a8_status s = device_info(&d)) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   EpilogueArgs ep;
   ep.S_x = S;
   ep.s_x_per_row = 0;
@@ -293,24 +335,36 @@ w8a8_status w8a8_linear_static(const void *X, int64_t M, int64_t K, int64_t ldx,
   ep.bias = bias;
   ep.out = out;
   ep.out_dtype = out_dtype;
-  if (decode_fuses_quant(M, N))  // one kernel: the GEMM quantizes each k-block
-    return from_cuda(launch_linear_static_decode(static_cast<const uint16_t *>(X), ldx, r, Z, Wq, M, N, K, ep,
-                                                 d->status, st));
-  if (M <= kDecodeMaxM) {
-    // Static quantization into the workspace, then the decode GEMM; both use
-    // programmatic dependent launch, so the GEMM's weight stream starts while
-    // the quantization (and the previous kernel) run.
-    int8_t *Xq = static_cast<int8_t *>(workspace);
-    cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq, d->sm_count, st,
-                                            /*pdl=*/true);
-    if (e != cudaSuccess) return W8A8_ERR_CUDA;
-    return from_cuda(launch_gemm_decode(Xq, K, Wq, M, N, K, ep, d->status, st));
-  }
-  int8_t *Xq = static_cast<int8_t *>(workspace);
-  cudaError_t e = launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq,
-                                          d->sm_count, st, /*pdl=*/true);
-  if (e != cudaSuccess) return W8A8_ERR_CUDA;
-  return from_cuda(launch_gemm_tc(Xq, Wq, M, N, K, ep, false, d->sm_count, d->status, st));
+  return run_linear_static(X, M, K, ldx, r, Z, Wq, N, ep, workspace, workspace_bytes,
+                           static_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_linear_static_requant(const void *X, int64_t M, int64_t K, int64_t ldx, const float *S,
+                                       const float *r, const int32_t *Z, const int8_t *Wq,
+                                       const float *s_w, const int32_t *colsum, const float *bias,
+                                       int64_t N, const float *r_out, const int32_t *Z_out, int8_t *Xq_out,
+                                       void *workspace, size_t workspace_bytes, void *stream) {
+  if (w8a8_status s = check_bf16_rows(X, M, K, ldx)) return s;
+  if (N < 0) return W8A8_ERR_INVALID_ARG;
+  if (M > kDecodeMaxM) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if (!S || !r || !Z || !Wq || !s_w || !colsum || !r_out || !Z_out || !Xq_out) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(Wq) || !aligned16(s_w) || !aligned16(colsum) || !aligned16(Xq_out) ||
+      (bias && !aligned16(bias)))
+    return W8A8_ERR_MISALIGNED;
+  EpilogueArgs ep;
+  ep.S_x = S;
+  ep.s_x_per_row = 0;
+  ep.Z = Z;
+  ep.colsum = colsum;
+  ep.s_w = s_w;
+  ep.bias = bias;
+  ep.out = Xq_out;
+  ep.out_dtype = kOutRequantI8;
+  ep.r_out = r_out;
+  ep.z_out = Z_out;
+  return run_linear_static(X, M, K, ldx, r, Z, Wq, N, ep, workspace, workspace_bytes,
+                           static_cast<cudaStream_t>(stream));
 }
 
 size_t int8_outlier_split_workspace_size(int64_t K) {

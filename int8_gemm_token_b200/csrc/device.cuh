@@ -334,22 +334,24 @@ __device__ __forceinline__ uint2 quant8_sym_sat(const uint4 &v, float r) {
   return make_uint2(pack_sat_s8x4(q[0], q[1], q[2], q[3]), pack_sat_s8x4(q[4], q[5], q[6], q[7]));
 }
 
-// Static asymmetric codes: clamp(rne(x * r) + Z, -128, 127), with the rounded
-// value first held to [-1024, 1024] (invisible after the final clamp, since
-// |Z| <= 255) so that nothing overflows. Everything runs on the full-rate FP32
-// and integer pipes: adding 1.5 * 2^23 to a value of magnitude <= 2^22 leaves
-// it rounded to the nearest integer, ties to even, in the low mantissa bits.
 // Low bytes of four int32, a in the lowest byte.
 __device__ __forceinline__ uint32_t pack_i8x4(int a, int b, int c, int d) {
   return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
          ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
 }
 
+// rne(y) held to [-1024, 1024] on the full-rate FP32 and integer pipes: adding
+// 1.5 * 2^23 to a value of magnitude <= 2^22 leaves it rounded to the nearest
+// integer, ties to even, in the low mantissa bits.
 __device__ __forceinline__ int rne_held(float y) {
   y = fminf(fmaxf(y, -1024.0f), 1024.0f);
   return __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
 }
 
+// Static asymmetric codes of the 8 bf16 values in one uint4:
+// clamp(rne(x * r) + Z, -128, 127). Holding the rounded value to
+// [-1024, 1024] first is invisible after the final clamp (|Z| <= 255) and
+// keeps the sum from overflowing.
 __device__ __forceinline__ uint2 quant8_asym_sat(const uint4 &v, float r, int z) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   int q[8];

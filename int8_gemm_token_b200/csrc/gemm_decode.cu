@@ -35,7 +35,8 @@
 //     (st.shared::cluster). After one cluster barrier all 256 threads add the
 //     SPLIT partials (exact int32) of chunks of 8 outputs, run the epilogue
 //     with the per-channel constants fetched before the barrier, and store 16
-//     bytes at a time. No global workspace, no atomics;
+//     bytes at a time (8 when the epilogue writes the next linear's int8
+//     codes of the bf16 result instead). No global workspace, no atomics;
 //   * programmatic dependent launch: the kernel lets its dependents launch
 //     as soon as it has started, and requests its first ring of weight tiles
 //     before it waits for the previous kernel in the stream
@@ -149,8 +150,11 @@ __device__ __forceinline__ void load_consts8(const EpilogueArgs &ep, int64_t n0,
 // The epilogue of 8 consecutive outputs out[m, n0 .. n0+7] (n0 a multiple of
 // 8), each in the fixed order of include/w8a8.h:
 // c = acc - Z*colsum[n]; y = fmaf(float(c), S_x[m]*s_w[n], bias[n]).
+// kOutRequantI8 stores the next linear's static code of bf16(y) instead, with
+// its scalars rq = r_out and zq = Z_out.
 __device__ __forceinline__ void epilogue8(const EpilogueArgs &ep, int64_t m, int64_t n0, int64_t N,
-                                          const int32_t (&a)[8], int32_t z, float sx, const Consts8 &k) {
+                                          const int32_t (&a)[8], int32_t z, float sx, const Consts8 &k,
+                                          float rq, int32_t zq) {
   const bool full = n0 + 8 <= N;
   int32_t c[8];
   float y[8];
@@ -178,6 +182,21 @@ __device__ __forceinline__ void epilogue8(const EpilogueArgs &ep, int64_t m, int
           __nv_bfloat16 b = __float2bfloat16_rn(y[i]);
           out[i] = *reinterpret_cast<uint16_t *>(&b);
         }
+    }
+  } else if (ep.out_dtype == kOutRequantI8) {
+    uint4 v;  // bf16(y), exactly as the bf16 output stores it
+    v.x = pack_bf16x2(y[0], y[1]);
+    v.y = pack_bf16x2(y[2], y[3]);
+    v.z = pack_bf16x2(y[4], y[5]);
+    v.w = pack_bf16x2(y[6], y[7]);
+    const uint2 q = quant8_asym_sat(v, rq, zq);
+    int8_t *out = static_cast<int8_t *>(ep.out) + o;
+    if (full && (o % 8) == 0) {
+      *reinterpret_cast<uint2 *>(out) = q;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (n0 + i < N) out[i] = static_cast<int8_t>(((i < 4 ? q.x : q.y) >> (8 * (i & 3))) & 0xFFu);
     }
   } else if (ep.out_dtype == W8A8_FP32) {
     float *out = static_cast<float *>(ep.out) + o;
@@ -466,6 +485,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const int per_m = (owner_row0<SPLIT>(static_cast<int>(rank) + 1) - r0) / 8;
   const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
   const float sx0 = ep.s_x_per_row ? 0.0f : __ldg(ep.S_x);
+  const bool requant = ep.out_dtype == kOutRequantI8;
+  const float rq = requant ? __ldg(ep.r_out) : 0.0f;
+  const int32_t zq = requant ? __ldg(ep.z_out) : 0;
   Consts8 k0;
   {
     const int m = static_cast<int>(threadIdx.x) / per_m;
@@ -500,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         for (int i = 0; i < 8; ++i) a[i] += p[i];
       }
       const float sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : sx0;
-      epilogue8(ep, m, n0, N, a, z, sx, kc);
+      epilogue8(ep, m, n0, N, a, z, sx, kc, rq, zq);
     }
   }
 

@@ -29,8 +29,13 @@ struct EpilogueArgs {
   int64_t ldw = 0;
   // output
   void *out = nullptr;  // [M, N] dense
-  int32_t out_dtype = W8A8_BF16;
+  int32_t out_dtype = W8A8_BF16;  // a public w8a8_dtype, or kOutRequantI8
+  // kOutRequantI8 (Decode-shaped GEMM only): out is int8, the next linear's
+  // static code of the bf16 result, clamp(rne(bf16(y) * r_out) + Z_out, -128, 127)
+  const float *r_out = nullptr;    // device scalar
+  const int32_t *z_out = nullptr;  // device scalar
 };
+constexpr int32_t kOutRequantI8 = 16;  // internal; not a public dtype code
 
 // Once per kernel and device: raise the kernel's dynamic shared-memory limit to
 // at least `bytes` (and ask for the largest shared-memory carveout). Later

@@ -45,6 +45,9 @@ _SIGNATURES = {
     "w8a8_gemm_dequant": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I32, _P, _SZ, _P]),
     "w8a8_gemm_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "w8a8_linear_static": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _SZ, _P]),
+    "w8a8_gemm_requant": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P]),
+    "w8a8_linear_static_requant": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _P,
+                                          _SZ, _P]),
     "w8a8_linear_static_noalloc": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P]),
     "int8_outlier_split": (_I32, [_P, _I64, _I64, _I64, _F, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "int8_outlier_split_workspace_size": (_SZ, [_I64]),
@@ -204,6 +207,35 @@ def w8a8_linear_static(X, S, r, Z, Wq, s_w, colsum, bias=None, out=None, out_dty
     _check("w8a8_linear_static", lib().w8a8_linear_static(
         _ptr(X), M, K, _ld(X), _ptr(S), _ptr(r), _ptr(Z), _ptr(Wq), _ptr(s_w), _ptr(colsum),
         _ptr(bias), N, _ptr(out), _dt(out.dtype), _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def w8a8_gemm_requant(Xq, S_x, Wq, s_w, r_out, Z_out, colsum=None, Z=None, bias=None, out=None, stream=None):
+    """w8a8_gemm_dequant whose bf16 result is quantized at once with the next
+    linear's static r_out, Z_out: returns int8 [M, N] (M <= 64)."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    out = torch.empty((M, N), dtype=torch.int8, device=Xq.device) if out is None else out
+    if S_x.numel() not in (1, M):
+        raise ValueError("S_x holds one scale per row or a single per-tensor scale")
+    per_row = 1 if S_x.numel() == M else 0
+    _check("w8a8_gemm_requant", lib().w8a8_gemm_requant(
+        _ptr(Xq), _ptr(S_x), per_row, _ptr(Z), _ptr(Wq), _ptr(s_w), _ptr(colsum), _ptr(bias), M, N, K,
+        _ptr(r_out), _ptr(Z_out), _ptr(out), _stream(stream)))
+    return out
+
+
+def w8a8_linear_static_requant(X, S, r, Z, Wq, s_w, colsum, r_out, Z_out, bias=None, out=None, workspace=None,
+                               stream=None):
+    """Decode linear whose bf16 result is quantized at once with the next
+    linear's static r_out, Z_out: returns int8 [M, N] (M <= 64)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    out = torch.empty((M, N), dtype=torch.int8, device=X.device) if out is None else out
+    ws, nbytes = _workspace(w8a8_gemm_workspace_size(M, N, K), X.device, workspace)
+    _check("w8a8_linear_static_requant", lib().w8a8_linear_static_requant(
+        _ptr(X), M, K, _ld(X), _ptr(S), _ptr(r), _ptr(Z), _ptr(Wq), _ptr(s_w), _ptr(colsum), _ptr(bias), N,
+        _ptr(r_out), _ptr(Z_out), _ptr(out), _ptr(ws), nbytes, _stream(stream)))
     return out
 
 

@@ -241,6 +241,19 @@ def linear_decode(X, r, Z, S, Wq, s_w, colsum, bias=None):
     return Xq, acc, y
 
 
+def linear_decode_requant(X, r, Z, S, Wq, s_w, colsum, r_out, Z_out, bias=None):
+    """PDMIX decode linear whose bf16 result is quantized for the next linear
+    with that linear's static r_out, Z_out (PDMIX glossary §2.3 eq. Q_decode
+    applied to the next layer's input). The result passes between layers as
+    bf16, so the code is taken from the bf16-rounded value.
+
+    Returns (Xq, acc, y_f32, y_bf16, Xq_out)."""
+    Xq, acc, y = linear_decode(X, r, Z, S, Wq, s_w, colsum, bias=bias)
+    y_bf16 = f32_to_bf16(y)
+    Xq_out = quant_per_tensor(y_bf16, r_out, Z_out)
+    return Xq, acc, y, y_bf16, Xq_out
+
+
 def linear_mixed(X, W_bf16, Wq, s_w, threshold=6.0, cap=64, bias=None):
     """LLM.int8() vector-wise INT8 path plus the 16-bit outlier side path.
 

@@ -78,6 +78,31 @@ def test_linear_static_workspace_check(L):
     assert f(GOOD, 4, 64, 64, GOOD, GOOD, None, GOOD, GOOD, GOOD, None, 8, GOOD, 0, GOOD, 4096, None) == 1
 
 
+def test_requant_entry_points_host_checks(L):
+    f = L.w8a8_linear_static_requant
+    # X, M, K, ldx, S, r, Z, Wq, s_w, colsum, bias, N, r_out, Z_out, Xq_out, ws, wsb, stream
+    base = [GOOD, 8, 64, 64, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, None, 8, GOOD, GOOD, GOOD, None, 0, None]
+
+    def call(**kw):
+        a = list(base)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+    assert call(a1=65) == 3                      # Decode-shaped only: M <= 64
+    assert call(a1=0) == 0 and call(a11=0) == 0
+    assert call(a12=None) == 1 and call(a13=None) == 1 and call(a14=None) == 1
+    assert call(a14=ODD) == 2
+    assert call(a1=40) == 9                      # 40 tokens: the workspace holds the quantized activation
+    g = L.w8a8_gemm_requant
+    # Xq, S_x, per_row, Z, Wq, s_w, colsum, bias, M, N, K, r_out, Z_out, Xq_out, stream
+    assert g(GOOD, GOOD, 0, GOOD, GOOD, GOOD, GOOD, None, 65, 8, 64, GOOD, GOOD, GOOD, None) == 3
+    assert g(GOOD, GOOD, 0, GOOD, GOOD, GOOD, GOOD, None, 8, 8, 40, GOOD, GOOD, GOOD, None) == 3
+    assert g(GOOD, GOOD, 0, GOOD, GOOD, GOOD, GOOD, None, 8, 8, 64, None, GOOD, GOOD, None) == 1
+    assert g(GOOD, GOOD, 0, GOOD, GOOD, GOOD, None, None, 8, 8, 64, GOOD, GOOD, GOOD, None) == 1  # Z without colsum
+    assert g(GOOD, GOOD, 0, GOOD, GOOD, GOOD, GOOD, None, 8, 8, 64, GOOD, GOOD, ODD, None) == 2
+    assert g(GOOD, GOOD, 0, GOOD, GOOD, GOOD, GOOD, None, 0, 8, 64, GOOD, GOOD, GOOD, None) == 0
+
+
 def test_other_entry_points_host_checks(L):
     assert L.w8a8_quant_weight_per_channel(GOOD, 5, 64, 8, 8, GOOD, GOOD, GOOD, None) == 4
     assert L.w8a8_quant_weight_per_channel(GOOD, 1, 64, 8, 4, GOOD, GOOD, GOOD, None) == 1
@@ -104,6 +129,7 @@ def test_valid_call_without_a_gpu_reports_no_device(L):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert L.w8a8_quant_per_token(GOOD, 4, 32, 32, GOOD, GOOD, None) == 10
+    assert L.w8a8_gemm_requant(GOOD, GOOD, 0, GOOD, GOOD, GOOD, GOOD, None, 8, 8, 64, GOOD, GOOD, GOOD, None) == 10
     assert w8a8.w8a8_gemm_workspace_size(4, 8, 64) == 0  # one kernel: quantized inside the GEMM
     assert w8a8.w8a8_gemm_workspace_size(32, 4096, 64) == 0
     assert w8a8.w8a8_gemm_workspace_size(32, 4104, 64) >= 32 * 64  # quantization kernel first

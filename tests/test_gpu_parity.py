@@ -344,3 +344,113 @@ def test_decode_linear_static_every_finite_bf16_activation(M, N):
     rwq, rws, rwc = oracle.quant_weight_per_channel(case.W)
     _, _, y = oracle.linear_decode(X, rr, rZ, rS, rwq, rws, rwc)
     assert_same(host(out), y, "out")
+
+
+# ------------------------------------------------------------ static requantization for the next linear
+
+
+def _next_linear_params(y_bf16, shrink=0.7):
+    """The next linear's static (S, r, Z): the oracle's MinMax over this
+    layer's bf16 result, the range narrowed so that both ends saturate."""
+    yf = oracle.bf16_to_f32(y_bf16)
+    cal = oracle.f32_to_bf16(np.clip(yf, shrink * yf.min(), shrink * yf.max()))
+    return oracle.calibrate_static(cal)
+
+
+@pytest.mark.parametrize("M,N,K,ld_pad", [(1, 4096, 4096, 0), (16, 11008, 4096, 0), (32, 4096, 4096, 0),
+                                          (32, 11008, 4096, 0), (3, 1001, 400, 8), (48, 300, 400, 8),
+                                          (64, 520, 2048, 0), (24, 5000, 1024, 0), (33, 4104, 512, 0)])
+def test_decode_requant_bit_exact(M, N, K, ld_pad):
+    """w8a8_linear_static_requant: the next linear's int8 codes of this
+    linear's bf16 result equal the oracle's, in the one-kernel form (M <= 16,
+    or M <= 32 with N <= 4096) and with the separate quantization kernel, on
+    ragged N (rows of Xq_out not 8-byte aligned) and padded activation rows."""
+    case = synth.decode_static(M=M, N=N, K=K, seed=3 * M + N)
+    rS, rr, rZ = oracle.calibrate_static(case.Xcal)
+    rwq, rws, rwc = oracle.quant_weight_per_channel(case.W)
+    bias = synth.bias(np.random.default_rng(2), N)
+    _, _, _, y_bf16, _ = oracle.linear_decode_requant(case.X, rr, rZ, rS, rwq, rws, rwc, np.float32(1), 0,
+                                                      bias=bias)
+    _, r2, Z2 = _next_linear_params(y_bf16)
+    q_ref = oracle.linear_decode_requant(case.X, rr, rZ, rS, rwq, rws, rwc, r2, Z2, bias=bias)[4]
+    assert (q_ref == 127).any() and (q_ref == -128).any()
+
+    S, r, Z = W.w8a8_calibrate_static(dev_bf16(case.Xcal))
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(case.W))
+    Xd = dev_bf16(np.pad(case.X, ((0, 0), (0, ld_pad))))[:, :K]
+    r2d = torch.tensor([r2], dtype=torch.float32, device="cuda")
+    Z2d = torch.tensor([Z2], dtype=torch.int32, device="cuda")
+    ws = W.new_workspace(M, N, K)
+    q = W.w8a8_linear_static_requant(Xd, S, r, Z, Wq, s_w, cs, r2d, Z2d, bias=dev(bias), workspace=ws)
+    assert q.dtype == torch.int8 and tuple(q.shape) == (M, N)
+    assert_same(host(q), q_ref, "Xq_out")
+    if N % 16 == 0:  # the same as the two calls it replaces (quantization rows are multiples of 16)
+        out = W.w8a8_linear_static(Xd, S, r, Z, Wq, s_w, cs, bias=dev(bias), workspace=ws)
+        assert torch.equal(q, W.w8a8_quant_per_tensor(out, r2d, Z2d))
+
+
+@pytest.mark.parametrize("graph", [False, True])
+def test_decode_requant_chain_of_linears(graph):
+    """Three Decode linears chained on one stream with no synchronization:
+    linear 1 quantizes bf16 X and hands int8 codes to linear 2
+    (w8a8_linear_static_requant), linear 2 takes codes and hands codes on
+    (w8a8_gemm_requant), linear 3 takes codes and writes bf16
+    (w8a8_gemm_dequant), each with its own static S, Z. Each kernel may start its weight stream while the previous
+    one runs; every result must equal the oracle's chain."""
+    M, widths = 32, [2048, 4096, 1024, 3000]
+    rng = np.random.default_rng(44)
+    Xcal = synth.calibration_tokens(rng, 256, widths[0])
+    X = synth.calibration_tokens(rng, M, widths[0])
+    Ws = [synth.weight(np.random.default_rng(50 + i), widths[i], widths[i + 1]) for i in range(3)]
+    # oracle chain; each next linear calibrated on the previous one's bf16 result
+    S1, r1, Z1 = oracle.calibrate_static(Xcal)
+    qs = [oracle.quant_weight_per_channel(w) for w in Ws]
+    y1 = oracle.linear_decode_requant(X, r1, Z1, S1, *qs[0], np.float32(1), 0)[3]
+    S2, r2, Z2 = _next_linear_params(y1, 0.8)
+    q1 = oracle.linear_decode_requant(X, r1, Z1, S1, *qs[0], r2, Z2)[4]
+    acc2 = oracle.gemm_i64(q1, qs[1][0])
+    y2 = oracle.f32_to_bf16(oracle.epilogue(acc2, np.float32(S2), qs[1][1], colsum=qs[1][2], Z=Z2))
+    S3, r3, Z3 = _next_linear_params(y2, 0.8)
+    q2 = oracle.quant_per_tensor(y2, r3, Z3)
+    y3 = oracle.f32_to_bf16(oracle.epilogue(oracle.gemm_i64(q2, qs[2][0]), np.float32(S3), qs[2][1],
+                                            colsum=qs[2][2], Z=Z3))
+
+    def scal(v, dt):
+        return torch.tensor([v], dtype=dt, device="cuda")
+    Xd = dev_bf16(X)
+    S1d, r1d, Z1d = W.w8a8_calibrate_static(dev_bf16(Xcal))
+    S2d, r2d, Z2d = scal(S2, torch.float32), scal(r2, torch.float32), scal(Z2, torch.int32)
+    S3d, r3d, Z3d = scal(S3, torch.float32), scal(r3, torch.float32), scal(Z3, torch.int32)
+    wd = [W.w8a8_quant_weight_per_channel(dev(w)) for w in Ws]
+    ws = W.new_workspace(M, max(widths), max(widths))
+    q1d = torch.empty((M, widths[1]), dtype=torch.int8, device="cuda")
+    q2d = torch.empty((M, widths[2]), dtype=torch.int8, device="cuda")
+    y3d = torch.empty((M, widths[3]), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+
+    def step():
+        W.w8a8_linear_static_requant(Xd, S1d, r1d, Z1d, *wd[0], r2d, Z2d, out=q1d, workspace=ws)
+        W.w8a8_gemm_requant(q1d, S2d, wd[1][0], wd[1][1], r3d, Z3d, colsum=wd[1][2], Z=Z2d, out=q2d)
+        W.w8a8_gemm_dequant(q2d, S3d, wd[2][0], wd[2][1], colsum=wd[2][2], Z=Z3d, out=y3d)
+
+    if graph:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            step()
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        q1d.fill_(-99)  # the replay must rewrite every output
+        q2d.fill_(-99)
+        y3d.fill_(float("nan"))
+        g.replay()
+        g.replay()
+    else:
+        step()
+        step()
+    torch.cuda.synchronize()
+    assert_same(host(q1d), q1, "codes for linear 2")
+    assert_same(host(q2d), q2, "codes for linear 3")
+    assert_same(host_bf16(y3d), y3, "linear 3")

@@ -262,6 +262,32 @@ def test_decode_layer_error_bound():
     assert np.all(np.abs(y - ref) <= bound)
 
 
+def test_decode_requant_of_a_hand_worked_layer():
+    """Static requantization for the next linear, worked by hand. With S = 1,
+    r = 1, Z = 0 the activation codes are the integers of X; one channel of
+    ones over the first three inputs gives y = 127 + 127 + 7 = 261. bf16 keeps
+    8 significant bits, so 261 is stored as 260; with r_out = 1, Z_out = -200
+    the code is 260 - 200 = 60 (quantizing the fp32 value would give 61, and
+    dropping Z_out would saturate at 127). A second channel of -1s gives
+    y = -261 -> bf16 -260 -> -460, saturated to -128."""
+    K = 16
+    X = np.zeros((1, K), np.float32)
+    X[0, :3] = [127.0, 127.0, 7.0]
+    Wq = np.zeros((2, K), np.int8)
+    Wq[0, :3] = 1
+    Wq[1, :3] = -1
+    s_w = np.ones(2, np.float32)
+    colsum = Wq.astype(np.int32).sum(1).astype(np.int32)
+    _, acc, y, y_bf16, q = oracle.linear_decode_requant(bf(X), F32(1.0), 0, F32(1.0), Wq, s_w, colsum,
+                                                        F32(1.0), -200)
+    assert acc.tolist() == [[261, -261]] and y.tolist() == [[261.0, -261.0]]
+    assert f32(y_bf16).tolist() == [[260.0, -260.0]]
+    assert q.tolist() == [[60, -128]]
+    # a scaled case: r_out = 0.25 maps bf16 260 to 65 exactly; Z_out = 3 shifts it
+    q2 = oracle.linear_decode_requant(bf(X), F32(1.0), 0, F32(1.0), Wq, s_w, colsum, F32(0.25), 3)[4]
+    assert q2.tolist() == [[68, -62]]
+
+
 def test_epilogue_fixed_order():
     """fmaf(float(c), S_x*s_w, side + bias) with single roundings, checked
     against float64 evaluation of the same expression rounded once."""
