@@ -332,6 +332,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.empty_cache()
     # ---------------------------------------------------------------- the other rows of the path
     decode = llm = block = None
+    quant_stream = bench_quant_stream(dev, peaks)
     if not args.no_decode:
         decode = bench_decode(args, dev, rank, peaks)
     if not args.no_llm_int8:
@@ -363,7 +364,8 @@ def run_ours(args, world, rank, local):
                          "algorithmic_bytes": M * K + N * K + 2 * M * N + 4 * M + 8 * N},
             "quant": {"kernel": "quant_per_token_kernel", "ms": quant_ms, "achieved": quant_gbs,
                       "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": quant_gbs / peaks["hbm_gbs"],
-                      "C_s_over_C_g": quant_ms / gemm_ms},
+                      "C_s_over_C_g": quant_ms / gemm_ms, "timing": "events around each launch in the step",
+                      "stream": quant_stream},
             "gemm_ms": gemm_ms,
             "decode": decode,
             "llm_int8": llm,
@@ -406,6 +408,38 @@ def graph_time_us(fn, n_calls, reps=10):
     torch.cuda.synchronize()
     del g
     return a.elapsed_time(b) * 1e3 / (reps * n_calls)
+
+
+def bench_quant_stream(dev, peaks):
+    """Per-token quantization alone: per-launch device time of back-to-back
+    launches in a CUDA graph, inputs and outputs rotated over > 2x L2, at the
+    step's shape and at the block's widest input (4096 tokens x 11008). One
+    event pair around a single 25 MB launch mostly measures its launch and
+    ramp; this measures the kernel's streaming rate."""
+    import torch
+
+    from int8_gemm_token_b200 import w8a8 as W
+    rows = []
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    for (Mq, Kq) in ((M, K), (4096, 11008)):
+        per = 3.0 * Mq * Kq
+        n = max(3, int(400e6 // per) + 1)
+        # rows of N(0,1) scaled by exp(N(0, 0.5)), as the step's activations
+        X0 = (torch.randn((Mq, Kq), device=dev, generator=g)
+              * torch.exp(0.5 * torch.randn((Mq, 1), device=dev, generator=g))).to(torch.bfloat16)
+        Xs = [X0.clone() for _ in range(n)]
+        Xqs = [torch.empty((Mq, Kq), dtype=torch.int8, device=dev) for _ in range(n)]
+        Ss = [torch.empty((Mq,), dtype=torch.float32, device=dev) for _ in range(n)]
+        us = graph_time_us(lambda i: W.w8a8_quant_per_token(Xs[i % n], Xq=Xqs[i % n], S_x=Ss[i % n]), 2 * n)
+        nbytes = 2.0 * Mq * Kq + Mq * Kq + 4.0 * Mq
+        gbs = nbytes / (us * 1e-6) / 1e9
+        rows.append({"M": Mq, "K": Kq, "us": us, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]})
+        del Xs, Xqs, Ss, X0
+    torch.cuda.empty_cache()
+    return {"workload": "quant_per_token_kernel alone, back-to-back launches in a CUDA graph, inputs and outputs "
+                        "rotated over > 400 MB", "rows": rows, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+            "algorithmic_bytes": "2MK + MK + 4M per launch"}
 
 
 def bench_decode(args, dev, rank, peaks):
