@@ -189,6 +189,51 @@ def test_prefill_7b_full_size_sampled():
     assert_same(got, oracle.f32_to_bf16(y), "sampled out")
 
 
+def test_pdmix_block_full_size_sampled():
+    """The PDMIX block workload at full size, in the launch configuration the
+    benchmark times: for each of the four linears (QKV, O, gate+up, down), one
+    INT8 weight serves a 4096-token Prefill (per-token quant + GEMM) and
+    Decode steps of 32 tokens (static calibration + one fused call). Weights,
+    calibration scalars and the Decode outputs of the first and last step are
+    compared in full; Prefill codes, scales and outputs on sampled rows and
+    columns that the oracle computes one by one."""
+    rng = np.random.default_rng(123)
+    for L_ in synth.pdmix_block(seed=0):
+        what = f"{L_.name} {L_.K}->{L_.N}"
+        Wf = L_.weight()
+        Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(Wf))
+        rwq, rws, rwc = oracle.quant_weight_per_channel(Wf)
+        del Wf
+        assert_same(host(Wq), rwq, what + " Wq")
+        assert_same(host(s_w), rws, what + " s_w")
+        assert_same(host(cs), rwc, what + " colsum")
+        # Prefill, 4096 tokens
+        Xp = L_.prefill_input(4096)
+        Xq, S_x = W.w8a8_quant_per_token(dev_bf16(Xp))
+        out = W.w8a8_gemm_dequant(Xq, S_x, Wq, s_w)
+        rows = np.sort(rng.choice(4096, 48, replace=False))
+        rows[-1] = 4095
+        cols = np.sort(rng.choice(L_.N, 48, replace=False))
+        cols[-1] = L_.N - 1
+        rxq, rS = oracle.quant_per_token(Xp[rows])
+        assert_same(host(Xq)[rows], rxq, what + " Xq rows")
+        assert_same(host(S_x)[rows], rS, what + " S_x rows")
+        y = oracle.epilogue(oracle.gemm_i64(rxq, rwq[cols]), rS, rws[cols])
+        assert_same(host_bf16(out)[np.ix_(rows, cols)], oracle.f32_to_bf16(y), what + " prefill out")
+        del Xp, Xq, S_x, out
+        # Decode: calibration, then two of the 64 steps
+        cal = L_.calibration()
+        S, r, Z = W.w8a8_calibrate_static(dev_bf16(cal))
+        rS_t, rr, rZ = oracle.calibrate_static(cal)
+        assert (host(S)[0], host(r)[0], host(Z)[0]) == (rS_t, rr, rZ), what
+        work = W.new_workspace(32, L_.N, L_.K)
+        for step in (0, 63):
+            xd = L_.decode_input(step, 32)
+            o = W.w8a8_linear_static(dev_bf16(xd), S, r, Z, Wq, s_w, cs, workspace=work)
+            _, _, yd = oracle.linear_decode(xd, rr, rZ, rS_t, rwq, rws, rwc)
+            assert_same(host_bf16(o), oracle.f32_to_bf16(yd), f"{what} decode step {step}")
+
+
 # ------------------------------------------------------------ failure path
 def test_bounded_wait_reports_timeout_and_device_stays_usable():
     W.w8a8_debug_wait_timeout_selftest(2_000_000)
