@@ -332,7 +332,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.empty_cache()
     # ---------------------------------------------------------------- the other rows of the path
     decode = llm = block = None
-    quant_stream = bench_quant_stream(dev, peaks)
+    quant_stream = None if args.no_quant_stream else bench_quant_stream(dev, peaks)
     if not args.no_decode:
         decode = bench_decode(args, dev, rank, peaks)
     if not args.no_llm_int8:
@@ -620,6 +620,7 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-llm-int8", action="store_true")
     ap.add_argument("--no-block", action="store_true")
+    ap.add_argument("--no-quant-stream", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=16)
