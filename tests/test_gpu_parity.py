@@ -499,3 +499,25 @@ def test_decode_requant_chain_of_linears(graph):
     assert_same(host(q1d), q1, "codes for linear 2")
     assert_same(host(q2d), q2, "codes for linear 3")
     assert_same(host_bf16(y3d), y3, "linear 3")
+
+
+def test_gemm_requant_per_token_scales_and_bias():
+    """w8a8_gemm_requant with one scale per token (a per-token quantized
+    activation), no zero point and a bias: the codes equal the oracle's
+    epilogue -> bf16 -> static quantization, on a ragged N."""
+    M, N, K = 20, 1000, 512
+    rng = np.random.default_rng(31)
+    X = synth.activations(rng, M, K, with_outliers=True)
+    Wf = synth.weight(rng, K, N)
+    bias = synth.bias(rng, N)
+    rxq, rS = oracle.quant_per_token(X)
+    rwq, rws, _ = oracle.quant_weight_per_channel(Wf)
+    y_bf16 = oracle.f32_to_bf16(oracle.epilogue(oracle.gemm_i64(rxq, rwq), rS, rws, bias=bias))
+    _, r2, Z2 = _next_linear_params(y_bf16)
+    q_ref = oracle.quant_per_tensor(y_bf16, r2, Z2)
+    Xq, S_x = W.w8a8_quant_per_token(dev_bf16(X))
+    Wq, s_w, _ = W.w8a8_quant_weight_per_channel(dev(Wf))
+    r2d = torch.tensor([r2], dtype=torch.float32, device="cuda")
+    Z2d = torch.tensor([Z2], dtype=torch.int32, device="cuda")
+    q = W.w8a8_gemm_requant(Xq, S_x, Wq, s_w, r2d, Z2d, bias=dev(bias))
+    assert_same(host(q), q_ref, "Xq_out")
