@@ -53,6 +53,7 @@ def _load():
                 "oracle_quant_weight_per_channel": (None, [P, ctypes.c_int, I64, I64, I64, P, P, P]),
                 "oracle_calibrate_static": (None, [P, ctypes.c_int, I64, I64, I64, P, P, P]),
                 "oracle_quant_per_tensor": (None, [P, ctypes.c_int, I64, I64, I64, F, I32, P]),
+                "oracle_dequant_per_tensor": (None, [P, I64, I64, F, I32, ctypes.c_int, P]),
                 "oracle_gemm_i64": (None, [P, P, I64, I64, I64, P]),
                 "oracle_epilogue": (ctypes.c_int, [P, I64, I64, P, ctypes.c_int, P, P, P, P, P, P]),
                 "oracle_f32_to_bf16_array": (None, [P, I64, P]),
@@ -150,6 +151,15 @@ def quant_per_tensor(X: np.ndarray, r, Z):
     Xq = np.empty((M, K), dtype=np.int8)
     _load().oracle_quant_per_tensor(_ptr(X), _dtype_code(X), M, K, K, float(np.float32(r)), int(Z), _ptr(Xq))
     return Xq
+
+
+def dequant_per_tensor(Xq: np.ndarray, S, Z, out_dtype: int = DT_BF16) -> np.ndarray:
+    """Static dequantization x = S * (q - Z): bf16 bits (DT_BF16) or float32."""
+    Xq = _c(np.asarray(Xq, dtype=np.int8))
+    M, K = Xq.shape
+    out = np.empty((M, K), dtype=np.uint16 if out_dtype == DT_BF16 else np.float32)
+    _load().oracle_dequant_per_tensor(_ptr(Xq), M, K, float(np.float32(S)), int(Z), int(out_dtype), _ptr(out))
+    return out
 
 
 def gemm_i64(Xq: np.ndarray, Wq: np.ndarray) -> np.ndarray:

@@ -194,6 +194,25 @@ void oracle_quant_per_tensor(const void *X, int dtype, int64_t M, int64_t K, int
     }
 }
 
+/* Per-tensor static dequantization: x = S * (q - Z), the inverse that the
+ * linear quantizer q = round(x / S) + Z of glossary §2.3 implies (the same
+ * x ~ S (q - Z) the four-term expansion of the LLM.int8() summary §一.2
+ * expands). The difference q - Z is an exact small integer, so the only
+ * rounding is the one fp32 product; out_dtype 0 then rounds it to bf16. */
+void oracle_dequant_per_tensor(const int8_t *Xq, int64_t M, int64_t K, float S, int32_t Z, int out_dtype,
+                               void *out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) {
+            float y = S * (float)((int32_t)Xq[m * K + k] - Z);
+            if (out_dtype == 0)
+                ((uint16_t *)out)[m * K + k] = oracle_f32_to_bf16(y);
+            else
+                ((float *)out)[m * K + k] = y;
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Integer GEMM (C4): acc[m, n] = sum_k Xq[m, k] * Wq[n, k], int64.           */
 /* LLM.int8() summary step (3): INT8 x INT8 products accumulated in INT32.    */

@@ -41,6 +41,8 @@ MUTATIONS = {
     "side_weight_row_index": ("W[(int64_t)idx[j] * ldw + n]", "W[(int64_t)j * ldw + n]"),
     "outliers_kept_in_row_scale": ("if (skip && skip[i]) continue;", ""),
     "bf16_round_half_away": ("u += 0x7fffu + keep_lsb;", "u += 0x8000u;"),
+    "dequant_zero_point_added": ("float y = S * (float)((int32_t)Xq[m * K + k] - Z);",
+                                 "float y = S * (float)((int32_t)Xq[m * K + k] + Z);"),
     "weight_read_along_rows": ("absmax_quant_vector(W, dtype, n, ldw, K, NULL, Wq + n * K, 1, &s_w[n]);",
                                "absmax_quant_vector(W, dtype, n, 1, K, NULL, Wq + n * K, 1, &s_w[n]);"),
 }

@@ -161,6 +161,31 @@ def test_static_quant_saturates_outside_range():
     assert list(q[0]) == [127, -128, 127, -128, 127, -128]
 
 
+def test_static_dequant_inverts_the_static_quantizer():
+    """x = S (q - Z), the inverse of eq. Q_decode (the INT8 KV cache's read
+    side). Hand values: S = 0.5, Z = -128 maps codes -128, 0, 127 to 0, 64,
+    127.5. q = Z gives exactly 0. Every code equals the exact real product
+    (float64 holds it) rounded once to fp32, and bf16 output is torch's
+    rounding of that. Codes of calibrated values come back within S/2."""
+    hand = np.zeros((1, 16), np.int8)
+    hand[0, :3] = [-128, 0, 127]
+    y = oracle.dequant_per_tensor(hand, F32(0.5), -128, oracle.DT_FP32)
+    assert y[0, :3].tolist() == [0.0, 64.0, 127.5]
+    codes = np.arange(-128, 128).astype(np.int8)[None, :]
+    for S, Z in [(F32(0.5), -128), (F32(0.013), 7), (F32(3.0e-3), 127), (F32(250.0), -5)]:
+        y = oracle.dequant_per_tensor(codes, S, Z, oracle.DT_FP32)
+        exact = (float(S) * (codes.astype(np.float64) - Z)).astype(np.float32)
+        assert np.array_equal(y, exact)
+        assert y[0, Z + 128] == 0.0
+        assert np.array_equal(oracle.dequant_per_tensor(codes, S, Z), bf(exact))
+    rng = np.random.default_rng(12)
+    Xcal = synth.activations(rng, 32, 64)
+    S, r, Z = oracle.calibrate_static(Xcal)
+    q = oracle.quant_per_tensor(Xcal, r, Z)
+    back = oracle.dequant_per_tensor(q, S, Z, oracle.DT_FP32).astype(np.float64)
+    assert np.all(np.abs(f32(Xcal).astype(np.float64) - back) <= float(S) * (0.5 + 1e-4))
+
+
 def test_calibration_all_zero_is_identity_scale():
     S, r, Z = oracle.calibrate_static(bf(np.zeros((4, 16), np.float32)))
     assert (S, r, Z) == (1.0, 1.0, 0)
