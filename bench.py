@@ -66,7 +66,7 @@ TC2_TRAFFIC = {
     "bytes": 53_721_088 + 6_855_936,
     "sources": ["int8_gemm_token_b200/csrc/gemm_tc.cu", "int8_gemm_token_b200/csrc/device.cuh",
                 "int8_gemm_token_b200/csrc/kernels.h"],
-    "sources_sha256": "162deaec986b446b20d5d9bbdf721dbf707222c26f734c216e01986cf9b0fc16",
+    "sources_sha256": "618a36b4be796305069921bd1b280bbae5165deeef21cfa4452a7d6056deb35c",
     "profile": "profiles/gemm_i8_tc2_prefill_7b_2048x4096x11008.txt",
 }
 
@@ -331,10 +331,11 @@ def run_ours(args, world, rank, local):
     del sets
     torch.cuda.empty_cache()
     # ---------------------------------------------------------------- the other rows of the path
-    decode = llm = block = None
+    decode = llm = block = kv = None
     quant_stream = None if args.no_quant_stream else bench_quant_stream(dev, peaks)
     if not args.no_decode:
         decode = bench_decode(args, dev, rank, peaks)
+        kv = bench_kv_cache(dev, peaks)
     if not args.no_llm_int8:
         llm = bench_llm_int8(args, dev, rank, peaks, int8_peak)
     if not args.no_block:
@@ -368,6 +369,7 @@ def run_ours(args, world, rank, local):
                       "stream": quant_stream},
             "gemm_ms": gemm_ms,
             "decode": decode,
+            "kv_cache": kv,
             "llm_int8": llm,
             "pdmix_block": block,
             "cpu_baseline": cpu,
@@ -440,6 +442,38 @@ def bench_quant_stream(dev, peaks):
     return {"workload": "quant_per_token_kernel alone, back-to-back launches in a CUDA graph, inputs and outputs "
                         "rotated over > 400 MB", "rows": rows, "unit": "GB/s", "peak": peaks["hbm_gbs"],
             "algorithmic_bytes": "2MK + MK + 4M per launch"}
+
+
+def bench_kv_cache(dev, peaks):
+    """INT8 KV cache kept in the Decode scheme: writing one cache tensor
+    (bf16 -> codes, w8a8_quant_per_tensor) and reading it back (codes -> bf16,
+    w8a8_dequant_per_tensor), 8192 tokens x 4096 (32 heads x 128), back to
+    back in a CUDA graph over tensors rotated beyond L2."""
+    import torch
+
+    from int8_gemm_token_b200 import w8a8 as W
+    T, D = 8192, 4096
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    X0 = (torch.randn((T, D), device=dev, generator=g)
+          * torch.exp(0.5 * torch.randn((T, 1), device=dev, generator=g))).to(torch.bfloat16)
+    S, r, Z = W.w8a8_calibrate_static(X0[:512])
+    n = 4
+    Xs = [X0.clone() for _ in range(n)]
+    Qs = [W.w8a8_quant_per_tensor(x, r, Z) for x in Xs]
+    del X0
+    write_us = graph_time_us(lambda i: W.w8a8_quant_per_tensor(Xs[i % n], r, Z, Xq=Qs[i % n]), 2 * n)
+    read_us = graph_time_us(lambda i: W.w8a8_dequant_per_tensor(Qs[i % n], S, Z, out=Xs[i % n]), 2 * n)
+    nbytes = 3.0 * T * D
+    rows = []
+    for name, us in (("write (quant_per_tensor)", write_us), ("read (dequant_per_tensor)", read_us)):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        rows.append({"op": name, "tokens": T, "width": D, "us": us, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]})
+    del Xs, Qs
+    torch.cuda.empty_cache()
+    return {"workload": "INT8 KV cache tensor, 8192 tokens x 4096, static per-tensor scheme; graph-timed, "
+                        "4 rotating tensors (> 2x L2 with their codes)", "rows": rows, "unit": "GB/s",
+            "peak": peaks["hbm_gbs"], "algorithmic_bytes": "3 * tokens * width per call"}
 
 
 def bench_decode(args, dev, rank, peaks):

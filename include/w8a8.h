@@ -130,6 +130,25 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
                                   const int32_t *Z, int8_t *Xq, void *stream);
 
 /*
+ * Static per-tensor dequantization, the inverse of w8a8_quant_per_tensor:
+ *   out[m, k] = S * (float)(Xq[m, k] - Z)     (one fp32 product; q - Z is exact)
+ * rounded to bf16 (RNE) for W8A8_BF16, or stored as fp32 for W8A8_FP32.
+ * This is the read side of an INT8 KV cache kept in the Decode scheme: K and
+ * V quantized once with w8a8_calibrate_static's S, r, Z and
+ * w8a8_quant_per_tensor, and expanded by this call where attention needs
+ * them (attention itself is not part of this library).
+ * Source: PDMIX glossary §2.3 (q = round(x / S) + Z, so x ~ S (q - Z)) and
+ * §3 (KVCache Quant, the companion of PDMIX); PDMIX configuration guide (the
+ * W8A8C8 combination). No page fixes a separate scheme for the cache, so the
+ * Decode scheme is taken.
+ *   Xq   device int8 [M, K], row stride ldq bytes (a multiple of 16)
+ *   S, Z device scalars (fp32, int32), as from w8a8_calibrate_static
+ *   out  device [M, K] dense, 16-byte aligned, written
+ */
+w8a8_status w8a8_dequant_per_tensor(const int8_t *Xq, int64_t M, int64_t K, int64_t ldq, const float *S,
+                                    const int32_t *Z, void *out, w8a8_dtype out_dtype, void *stream);
+
+/*
  * INT8 x INT8 -> INT32 GEMM with the dequant epilogue fused in.
  * Source: LLM.int8() summary steps (3)-(4) (INT32 accumulation; rescale by
  * the outer product of the row and column constants) and §一.2 four-term

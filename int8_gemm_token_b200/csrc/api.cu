@@ -198,6 +198,21 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
                                            d->sm_count, static_cast<cudaStream_t>(stream)));
 }
 
+w8a8_status w8a8_dequant_per_tensor(const int8_t *Xq, int64_t M, int64_t K, int64_t ldq, const float *S,
+                                    const int32_t *Z, void *out, w8a8_dtype out_dtype, void *stream) {
+  if (M < 0) return W8A8_ERR_INVALID_ARG;
+  if (w8a8_status s = check_k(K)) return s;
+  if (ldq < K) return W8A8_ERR_INVALID_ARG;
+  if (out_dtype != W8A8_BF16 && out_dtype != W8A8_FP32) return W8A8_ERR_UNSUPPORTED_DTYPE;
+  if (M == 0) return W8A8_OK;
+  if (!Xq || !S || !Z || !out) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(Xq) || (ldq % 16) != 0 || !aligned16(out)) return W8A8_ERR_MISALIGNED;
+  DeviceInfo *d;
+  if (w8a8_status s = device_info(&d)) return s;
+  return from_cuda(launch_dequant_per_tensor(Xq, M, K, ldq, S, Z, out, out_dtype == W8A8_BF16, d->sm_count,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 // Calls with at most this many tokens take the weight-streaming decode kernel
 // (with the int8 activation); the one-kernel Decode linear serves up to 32.
 constexpr int64_t kDecodeMaxM = 64;

@@ -6,6 +6,8 @@
 //    into registers, absmax by warp shuffles, one fp32 division per row,
 //    quantize from registers, 8-byte int8 stores.
 //  * quant_per_tensor: PDMIX glossary §2.3 eq. Q_decode (static S, Z).
+//  * dequant_per_tensor: its inverse x = S (q - Z), the read side of an INT8
+//    KV cache kept in the Decode scheme.
 //  * calibrate_static: MinMax over all calibration elements (configuration
 //    guide Step 3: MinMax observer, asymmetric decode parameters).
 //  * quant_weight_per_channel: configuration guide Step 2 (int8 per_channel
@@ -152,6 +154,59 @@ cudaError_t launch_quant_per_tensor(const uint16_t *X, int64_t M, int64_t K, int
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, quant_per_tensor_kernel, X, M, K, ldx, r, Z, Xq);
+}
+
+// ------------------------------------------------------------ static dequantization
+// out[m, k] = S * float(Xq[m, k] - Z): one 16-byte load of 16 codes, one fp32
+// product each (q - Z is a small exact integer), 32 or 64 bytes stored.
+// Grid-stride over 16-code chunks; rows of Xq have stride ldq bytes.
+template <bool BF16_OUT>
+__global__ void __launch_bounds__(256) dequant_per_tensor_kernel(const int8_t *__restrict__ Xq, int64_t M,
+                                                                 int64_t K, int64_t ldq,
+                                                                 const float *__restrict__ S_ptr,
+                                                                 const int32_t *__restrict__ Z_ptr,
+                                                                 void *__restrict__ out) {
+  const float S = *S_ptr;
+  const int z = *Z_ptr;
+  const int64_t cpr = K >> 4;  // 16-code chunks per row
+  const int64_t total = M * cpr;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / cpr, c = i - m * cpr;
+    const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(Xq + m * ldq) + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float y[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int q = static_cast<int8_t>((w[j >> 2] >> (8 * (j & 3))) & 0xFFu);
+      y[j] = __fmul_rn(S, __int2float_rn(q - z));
+    }
+    if constexpr (BF16_OUT) {
+      uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + m * K) + 2 * c;
+      o[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                        pack_bf16x2(y[6], y[7]));
+      o[1] = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]), pack_bf16x2(y[12], y[13]),
+                        pack_bf16x2(y[14], y[15]));
+    } else {
+      float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + m * K) + 4 * c;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+    }
+  }
+}
+
+cudaError_t launch_dequant_per_tensor(const int8_t *Xq, int64_t M, int64_t K, int64_t ldq, const float *S,
+                                      const int32_t *Z, void *out, bool bf16_out, int num_sms, cudaStream_t s) {
+  const int64_t total = M * (K / 16);
+  int64_t blocks = (total + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
+  if (bf16_out)
+    dequant_per_tensor_kernel<true><<<grid, block, 0, s>>>(Xq, M, K, ldq, S, Z, out);
+  else
+    dequant_per_tensor_kernel<false><<<grid, block, 0, s>>>(Xq, M, K, ldq, S, Z, out);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------ calibration

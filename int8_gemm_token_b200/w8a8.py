@@ -42,6 +42,7 @@ _SIGNATURES = {
     "w8a8_calibrate_static": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]),
     "w8a8_quant_per_token": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "w8a8_quant_per_tensor": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _P]),
+    "w8a8_dequant_per_tensor": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P]),
     "w8a8_gemm_dequant": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I32, _P, _SZ, _P]),
     "w8a8_gemm_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "w8a8_linear_static": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _SZ, _P]),
@@ -156,6 +157,17 @@ def w8a8_quant_per_tensor(X: torch.Tensor, r: torch.Tensor, Z: torch.Tensor, Xq=
     _check("w8a8_quant_per_tensor", lib().w8a8_quant_per_tensor(
         _ptr(X), M, K, _ld(X), _ptr(r), _ptr(Z), _ptr(Xq), _stream(stream)))
     return Xq
+
+
+def w8a8_dequant_per_tensor(Xq: torch.Tensor, S: torch.Tensor, Z: torch.Tensor, out=None, out_dtype=torch.bfloat16,
+                            stream=None):
+    """int8 Xq [M, K] -> S * (Xq - Z) as bf16 or fp32 [M, K]."""
+    M, K = Xq.shape
+    out = torch.empty((M, K), dtype=out_dtype, device=Xq.device) if out is None else out
+    _check("w8a8_dequant_per_tensor", lib().w8a8_dequant_per_tensor(
+        _ptr(Xq), M, K, _ld(Xq), _ptr(S), _ptr(Z), _ptr(out), _dt(out.dtype),
+        _stream(stream)))
+    return out
 
 
 def w8a8_gemm_workspace_size(M: int, N: int, K: int) -> int:

@@ -111,6 +111,14 @@ def test_other_entry_points_host_checks(L):
     assert L.w8a8_calibrate_static(GOOD, 0, 0, 16, 16, GOOD, GOOD, GOOD, None) == 1
     assert L.w8a8_calibrate_static(GOOD, 3, 4, 16, 16, GOOD, GOOD, GOOD, None) == 4
     assert L.w8a8_quant_per_tensor(GOOD, 4, 64, 64, None, GOOD, GOOD, None) == 1
+    # Xq, M, K, ldq, S, Z, out, out_dtype, stream
+    assert L.w8a8_dequant_per_tensor(GOOD, 4, 40, 48, GOOD, GOOD, GOOD, 0, None) == 3    # K not a multiple of 16
+    assert L.w8a8_dequant_per_tensor(GOOD, 4, 64, 48, GOOD, GOOD, GOOD, 0, None) == 1    # ldq < K
+    assert L.w8a8_dequant_per_tensor(GOOD, 4, 64, 72, GOOD, GOOD, GOOD, 0, None) == 2    # rows not 16-byte aligned
+    assert L.w8a8_dequant_per_tensor(GOOD, 4, 64, 64, GOOD, GOOD, GOOD, 2, None) == 4    # no int32 output
+    assert L.w8a8_dequant_per_tensor(GOOD, 4, 64, 64, None, GOOD, GOOD, 0, None) == 1
+    assert L.w8a8_dequant_per_tensor(GOOD, 4, 64, 64, GOOD, GOOD, ODD, 1, None) == 2
+    assert L.w8a8_dequant_per_tensor(None, 0, 64, 64, None, None, None, 0, None) == 0
     assert L.int8_mixed_decomp_gemm(GOOD, GOOD, GOOD, GOOD, GOOD, 8, GOOD, GOOD, GOOD, 8, None,
                                     8, 8, 64, GOOD, 2, None) == 4  # int32 output not offered here
     assert L.int8_mixed_decomp_gemm(GOOD, GOOD, GOOD, GOOD, GOOD, 5000, GOOD, GOOD, GOOD, 8, None,

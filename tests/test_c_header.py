@@ -43,6 +43,7 @@ static int run_checks(void) {
   EXPECT(int8_mixed_decomp_gemm(P, P, P, P, P, 8, P, P, P, 8, NULL, 8, 8, 64, P, W8A8_I32, NULL),
          W8A8_ERR_UNSUPPORTED_DTYPE);
   EXPECT(w8a8_quant_weight_per_channel(P, 5, 64, 8, 8, P, P, P, NULL), W8A8_ERR_UNSUPPORTED_DTYPE);
+  EXPECT(w8a8_dequant_per_tensor(P, 4, 64, 64, P, P, P, W8A8_I32, NULL), W8A8_ERR_UNSUPPORTED_DTYPE);
   EXPECT(w8a8_check_device_error(NULL, NULL), W8A8_ERR_INVALID_ARG);
   if (strcmp(w8a8_status_string(W8A8_ERR_OUTLIER_OVERFLOW), "W8A8_ERR_OUTLIER_OVERFLOW") != 0) ++fails;
   if (strcmp(w8a8_status_string(12345), "W8A8_ERR_UNKNOWN") != 0) ++fails;

@@ -521,3 +521,37 @@ def test_gemm_requant_per_token_scales_and_bias():
     Z2d = torch.tensor([Z2], dtype=torch.int32, device="cuda")
     q = W.w8a8_gemm_requant(Xq, S_x, Wq, s_w, r2d, Z2d, bias=dev(bias))
     assert_same(host(q), q_ref, "Xq_out")
+
+
+# ------------------------------------------------------------ static dequantization (INT8 KV cache)
+
+
+@pytest.mark.parametrize("S,Z", [(0.5, -128), (0.013, 7), (3.0e-3, 127), (250.0, -5)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_dequant_every_code(S, Z, out_dtype):
+    """x = S (q - Z) for every int8 code, in rows with a padded stride."""
+    codes = np.tile(np.arange(-128, 128).astype(np.int8), (5, 2))  # [5, 512]
+    Xd = dev(np.pad(codes, ((0, 0), (0, 32))))[:, :512]
+    Sd = torch.tensor([S], dtype=torch.float32, device="cuda")
+    Zd = torch.tensor([Z], dtype=torch.int32, device="cuda")
+    got = W.w8a8_dequant_per_tensor(Xd, Sd, Zd, out_dtype=out_dtype)
+    if out_dtype == torch.bfloat16:
+        assert_same(host_bf16(got), oracle.dequant_per_tensor(codes, np.float32(S), Z), "bf16")
+    else:
+        assert_same(host(got), oracle.dequant_per_tensor(codes, np.float32(S), Z, oracle.DT_FP32), "fp32")
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (7, 4112), (4096, 4096), (333, 1024)])
+def test_kv_cache_round_trip(M, K):
+    """A KV-cache tensor quantized with the Decode scheme and read back:
+    the GPU's codes and bf16 values equal the oracle's."""
+    rng = np.random.default_rng(M + K)
+    cal = synth.activations(rng, 64, K, with_outliers=True)
+    X = synth.activations(rng, M, K, with_outliers=True)
+    S, r, Z = W.w8a8_calibrate_static(dev_bf16(cal))
+    q = W.w8a8_quant_per_tensor(dev_bf16(X), r, Z)
+    back = W.w8a8_dequant_per_tensor(q, S, Z)
+    rS, rr, rZ = oracle.calibrate_static(cal)
+    rq = oracle.quant_per_tensor(X, rr, rZ)
+    assert_same(host(q), rq, "codes")
+    assert_same(host_bf16(back), oracle.dequant_per_tensor(rq, rS, rZ), "values")
