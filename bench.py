@@ -66,7 +66,7 @@ TC2_TRAFFIC = {
     "bytes": 53_721_088 + 6_855_936,
     "sources": ["int8_gemm_token_b200/csrc/gemm_tc.cu", "int8_gemm_token_b200/csrc/device.cuh",
                 "int8_gemm_token_b200/csrc/kernels.h"],
-    "sources_sha256": "618a36b4be796305069921bd1b280bbae5165deeef21cfa4452a7d6056deb35c",
+    "sources_sha256": "096ffec6322f237f6f86bb5c0bf34b29db04a40caf89e568f7b5929ba55d2bee",
     "profile": "profiles/gemm_i8_tc2_prefill_7b_2048x4096x11008.txt",
 }
 

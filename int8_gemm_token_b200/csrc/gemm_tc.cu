@@ -8,18 +8,33 @@
 // the mixed mode the 16-bit decomposition step (2) and the final sum
 // Y = X_outlier W_outlier + Dequant(Q(X_normal) Q(W_normal)).
 //
-// How (sm_100a): one persistent CTA per SM walks output tiles of 128 x BN.
+// How (sm_100a): two persistent, warp-specialized kernels.
+//   gemm_i8_tc_kernel (fewer than 256 tokens): one CTA per SM walks output
+//   tiles of 128 x BN.
+//   gemm_i8_tc2_kernel (256 tokens and more): a cluster of two CTAs per pair
+//   of SMs walks 256 x 256 tiles; each CTA loads its own 128 rows of Xq and
+//   of Wq, the leader issues tcgen05.mma.cta_group::2 (M = 256) and commits
+//   to both CTAs' barriers, so each SM streams 2/3 of the operand bytes of a
+//   single-CTA tile. No load uses cluster multicast.
+// Roles in both:
 //   warp 0      TMA producer: 128-byte-swizzled K-major tiles of Xq [M, K]
 //               and Wq [N, K] into a STAGES-deep shared-memory ring;
 //   warp 1      TMEM allocator and MMA issuer: one thread issues
-//               tcgen05.mma (M=128, N=BN, K=32 bytes) into one of two TMEM
-//               accumulators (2 x BN int32 columns), tcgen05.commit frees
-//               ring slots and hands a finished accumulator to the epilogue;
-//   warps 4..7  epilogue: tcgen05.ld of the int32 accumulator (each warp its
-//               32-lane quarter), the fixed-order fp32 dequant, bf16 stores.
+//               tcgen05.mma (K = 32 bytes per instruction) into one of two
+//               TMEM accumulators, tcgen05.commit frees ring slots and hands
+//               a finished accumulator to the epilogue;
+//   warps 4..7  epilogue: the tile's per-column constants (s_w, 0 + bias,
+//               colsum) staged in shared memory while its MMAs run, then
+//               tcgen05.ld of the int32 accumulator (each warp its 32-lane
+//               quarter, the next 32 columns already in flight), the
+//               fixed-order fp32 dequant and bf16 / fp32 / int32 stores.
+//               The mixed (LLM.int8()) instantiation adds the 16-bit side
+//               product per element and keeps a serial per-chunk epilogue.
 // Double-buffered accumulators let the epilogue of tile i overlap the MMAs
-// of tile i+1. Every wait is bounded; on a timeout the CTA records
-// W8A8_ERR_DEVICE_TIMEOUT, stops, frees its TMEM and returns.
+// of tile i+1. Programmatic dependent launch: the first ring of weight tiles
+// is requested before griddepcontrol.wait, everything else after it. Every
+// wait is bounded; on a timeout the CTA records W8A8_ERR_DEVICE_TIMEOUT,
+// stops, frees its TMEM and returns.
 #include "device.cuh"
 #include "kernels.h"
 
