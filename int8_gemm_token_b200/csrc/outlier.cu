@@ -12,13 +12,18 @@
 // Pass 1 (column flags): each thread owns 8 adjacent columns (one 16-byte
 //   load per row) over a band of rows, keeps the largest magnitude per column
 //   and sets the columns' bits in a K-bit workspace bitmap when it exceeds the
-//   threshold (atomicOr only for outlier columns, so almost never).
-// Pass 2 (rows): every CTA turns the bitmap into the ascending index list
-//   (block-wide popcount scan, in shared memory); CTA 0 publishes it and the
-//   count. Each row is then loaded once into registers (16-byte loads),
-//   outlier columns are masked to zero, the absmax is reduced with warp
-//   shuffles, the row is quantized from registers, and the row's outlier
-//   values are gathered into Xo.
+//   threshold (atomicOr only for outlier columns, so almost never). X is
+//   loaded under an L2 evict-last policy so that pass 2 finds it in L2.
+// Pass 2 (rows): a grid sized to fill the SMs once; every CTA turns the
+//   bitmap into the ascending index list (block-wide popcount scan) and
+//   copies the bitmap into shared memory once; CTA 0 publishes the list and
+//   the count. The CTA then walks rows with a grid stride: each row is
+//   loaded once into registers (16-byte loads), with the next row's loads in
+//   flight when two rows fit in registers, outlier columns are masked to zero, the absmax is reduced with
+//   warp shuffles, the row is quantized from registers, and the row's
+//   outlier values are gathered into Xo. Pass 2 is launched with
+//   programmatic dependent launch and issues its first row loads before it
+//   waits for pass 1 (X is not written by pass 1).
 #include "device.cuh"
 #include "kernels.h"
 
