@@ -113,6 +113,14 @@ def _ld(t: torch.Tensor) -> int:
     return t.stride(0)
 
 
+def _expect(t: torch.Tensor, dtype, shape, what: str):
+    """Raise before the C call when a tensor the C side takes as a raw
+    pointer of a fixed type and dense layout is not that."""
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{what}: expected a contiguous {dtype} tensor of shape {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)}")
+
+
 # --------------------------------------------------------------------------
 # Entry points (same names as the C ABI)
 # --------------------------------------------------------------------------
@@ -163,7 +171,12 @@ def w8a8_dequant_per_tensor(Xq: torch.Tensor, S: torch.Tensor, Z: torch.Tensor, 
                             stream=None):
     """int8 Xq [M, K] -> S * (Xq - Z) as bf16 or fp32 [M, K]."""
     M, K = Xq.shape
+    if Xq.dtype != torch.int8:
+        raise ValueError(f"Xq: expected int8 codes, got {Xq.dtype}")
     out = torch.empty((M, K), dtype=out_dtype, device=Xq.device) if out is None else out
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError(f"out: expected bfloat16 or float32, got {out.dtype}")
+    _expect(out, out.dtype, (M, K), "out")
     _check("w8a8_dequant_per_tensor", lib().w8a8_dequant_per_tensor(
         _ptr(Xq), M, K, _ld(Xq), _ptr(S), _ptr(Z), _ptr(out), _dt(out.dtype),
         _stream(stream)))
@@ -227,7 +240,10 @@ def w8a8_gemm_requant(Xq, S_x, Wq, s_w, r_out, Z_out, colsum=None, Z=None, bias=
     linear's static r_out, Z_out: returns int8 [M, N] (M <= 64)."""
     M, K = Xq.shape
     N = Wq.shape[0]
+    _expect(Xq, torch.int8, (M, K), "Xq")
+    _expect(Wq, torch.int8, (N, K), "Wq")
     out = torch.empty((M, N), dtype=torch.int8, device=Xq.device) if out is None else out
+    _expect(out, torch.int8, (M, N), "out")
     if S_x.numel() not in (1, M):
         raise ValueError("S_x holds one scale per row or a single per-tensor scale")
     per_row = 1 if S_x.numel() == M else 0
@@ -243,7 +259,11 @@ def w8a8_linear_static_requant(X, S, r, Z, Wq, s_w, colsum, r_out, Z_out, bias=N
     linear's static r_out, Z_out: returns int8 [M, N] (M <= 64)."""
     M, K = X.shape
     N = Wq.shape[0]
+    if X.dtype != torch.bfloat16:
+        raise ValueError(f"X: expected bfloat16, got {X.dtype}")
+    _expect(Wq, torch.int8, (N, K), "Wq")
     out = torch.empty((M, N), dtype=torch.int8, device=X.device) if out is None else out
+    _expect(out, torch.int8, (M, N), "out")
     ws, nbytes = _workspace(w8a8_gemm_workspace_size(M, N, K), X.device, workspace)
     _check("w8a8_linear_static_requant", lib().w8a8_linear_static_requant(
         _ptr(X), M, K, _ld(X), _ptr(S), _ptr(r), _ptr(Z), _ptr(Wq), _ptr(s_w), _ptr(colsum), _ptr(bias), N,

@@ -144,3 +144,26 @@ def test_valid_call_without_a_gpu_reports_no_device(L):
     assert w8a8.w8a8_gemm_workspace_size(48, 100, 64) >= 48 * 64  # 33..64 tokens: quantization kernel first
     assert w8a8.w8a8_gemm_workspace_size(64, 8, 64) >= 64 * 64
     assert w8a8.lib().int8_outlier_split_workspace_size(8192) >= 8192 // 8
+
+
+def test_binding_rejects_wrong_output_types_before_the_c_call():
+    """The requantizing and dequantizing entry points take raw int8 / bf16 /
+    fp32 pointers; the binding refuses a tensor of another type or shape
+    before calling into the library (CPU tensors: nothing reaches a GPU)."""
+    import torch
+    Xq = torch.zeros((4, 32), dtype=torch.int8)
+    Wq = torch.zeros((8, 32), dtype=torch.int8)
+    s = torch.ones(1)
+    z = torch.zeros(1, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        w8a8.w8a8_gemm_requant(Xq, s, Wq, torch.ones(8), s, z, out=torch.zeros((4, 8), dtype=torch.float32))
+    with pytest.raises(ValueError):
+        w8a8.w8a8_gemm_requant(Xq, s, Wq, torch.ones(8), s, z, out=torch.zeros((4, 9), dtype=torch.int8))
+    with pytest.raises(ValueError):
+        w8a8.w8a8_gemm_requant(Xq.float(), s, Wq, torch.ones(8), s, z)
+    with pytest.raises(ValueError):
+        w8a8.w8a8_linear_static_requant(torch.zeros((4, 32)), s, s, z, Wq, torch.ones(8), torch.zeros(8), s, z)
+    with pytest.raises(ValueError):
+        w8a8.w8a8_dequant_per_tensor(Xq.to(torch.int32), s, z)
+    with pytest.raises(ValueError):
+        w8a8.w8a8_dequant_per_tensor(Xq, s, z, out=torch.zeros((4, 32), dtype=torch.int32))
