@@ -116,9 +116,13 @@ def test_gemm_int32_accumulator_bit_exact(M, N, K):
 
 
 # M >= 256 takes the CTA-pair kernel: ragged last row and column tiles, K not a
-# multiple of the 128-byte k-block.
+# multiple of the 128-byte k-block. (2048, 20480, 512) has 8 x 80 = 640 pair
+# tiles, more than the GPU has clusters, so every cluster walks several tiles
+# through both TMEM accumulator slots and their phase flips; (1000, 18000, 208)
+# does the same with ragged edges.
 @pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 400), (200, 264, 512), (520, 5000, 400),
-                                   (520, 5400, 256), (520, 5800, 272), (200, 11008, 512), (100, 2000, 400)])
+                                   (520, 5400, 256), (520, 5800, 272), (200, 11008, 512), (100, 2000, 400),
+                                   (2048, 20480, 512), (1000, 18000, 208)])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_prefill_linear_bit_exact(M, N, K, out_dtype):
     X, Wf, b = _rand_case(M, N, K, 3 * M + N)
@@ -163,10 +167,12 @@ def test_decode_linear_static_bit_exact(M, N):
     assert_same(host_bf16(out), oracle.f32_to_bf16(y), "out")
 
 
-def test_prefill_7b_full_size_sampled():
+def test_prefill_7b_full_size():
     """The full 2048 x 4096 x 11008 workload in the launch configuration the
-    benchmark uses; Xq, S_x, Wq, s_w, colsum are compared in full, outputs on
-    a sample of 96 rows x 96 columns that the oracle computes one by one."""
+    benchmark uses (the CTA-pair kernel, 8 x 43 = 344 pair tiles over the
+    GPU's clusters, so every cluster runs several tiles through both
+    accumulator slots): codes, scales, weight and every output element
+    compared with the oracle."""
     case = synth.prefill_7b(0)
     Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev(case.W))
     Xq, S_x = W.w8a8_quant_per_token(dev_bf16(case.X))
@@ -178,26 +184,18 @@ def test_prefill_7b_full_size_sampled():
     assert_same(host(Wq), rwq, "Wq")
     assert_same(host(s_w), rws, "s_w")
     assert_same(host(cs), rwc, "colsum")
-    rng = np.random.default_rng(99)
-    rows = np.sort(rng.choice(2048, 96, replace=False))
-    rows[-1] = 2047
-    cols = np.sort(rng.choice(11008, 96, replace=False))
-    cols[-1] = 11007
-    acc = oracle.gemm_i64(rxq[rows], rwq[cols])
-    y = oracle.epilogue(acc, rS[rows], rws[cols], bias=case.bias[cols])
-    got = host_bf16(out)[np.ix_(rows, cols)]
-    assert_same(got, oracle.f32_to_bf16(y), "sampled out")
+    y = oracle.epilogue(oracle.gemm_i64(rxq, rwq), rS, rws, bias=case.bias)
+    assert_same(host_bf16(out), oracle.f32_to_bf16(y), "out")
 
 
-def test_pdmix_block_full_size_sampled():
+def test_pdmix_block_full_size():
     """The PDMIX block workload at full size, in the launch configuration the
     benchmark times: for each of the four linears (QKV, O, gate+up, down), one
     INT8 weight serves a 4096-token Prefill (per-token quant + GEMM) and
-    Decode steps of 32 tokens (static calibration + one fused call). Weights,
-    calibration scalars and the Decode outputs of the first and last step are
-    compared in full; Prefill codes, scales and outputs on sampled rows and
-    columns that the oracle computes one by one."""
-    rng = np.random.default_rng(123)
+    Decode steps of 32 tokens (static calibration + one call). Weights,
+    calibration scalars, Prefill codes, scales and every Prefill output
+    element, and every Decode output element of the first and last step, are
+    compared with the oracle."""
     for L_ in synth.pdmix_block(seed=0):
         what = f"{L_.name} {L_.K}->{L_.N}"
         Wf = L_.weight()
@@ -211,16 +209,12 @@ def test_pdmix_block_full_size_sampled():
         Xp = L_.prefill_input(4096)
         Xq, S_x = W.w8a8_quant_per_token(dev_bf16(Xp))
         out = W.w8a8_gemm_dequant(Xq, S_x, Wq, s_w)
-        rows = np.sort(rng.choice(4096, 48, replace=False))
-        rows[-1] = 4095
-        cols = np.sort(rng.choice(L_.N, 48, replace=False))
-        cols[-1] = L_.N - 1
-        rxq, rS = oracle.quant_per_token(Xp[rows])
-        assert_same(host(Xq)[rows], rxq, what + " Xq rows")
-        assert_same(host(S_x)[rows], rS, what + " S_x rows")
-        y = oracle.epilogue(oracle.gemm_i64(rxq, rwq[cols]), rS, rws[cols])
-        assert_same(host_bf16(out)[np.ix_(rows, cols)], oracle.f32_to_bf16(y), what + " prefill out")
-        del Xp, Xq, S_x, out
+        rxq, rS = oracle.quant_per_token(Xp)
+        assert_same(host(Xq), rxq, what + " Xq")
+        assert_same(host(S_x), rS, what + " S_x")
+        y = oracle.epilogue(oracle.gemm_i64(rxq, rwq), rS, rws)
+        assert_same(host_bf16(out), oracle.f32_to_bf16(y), what + " prefill out")
+        del Xp, Xq, S_x, out, rxq, y
         # Decode: calibration, then two of the 64 steps
         cal = L_.calibration()
         S, r, Z = W.w8a8_calibrate_static(dev_bf16(cal))
