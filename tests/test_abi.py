@@ -5,6 +5,7 @@ import ctypes
 import subprocess
 
 import pytest
+import torch
 
 from int8_gemm_token_b200 import w8a8
 
@@ -167,3 +168,58 @@ def test_binding_rejects_wrong_output_types_before_the_c_call():
         w8a8.w8a8_dequant_per_tensor(Xq.to(torch.int32), s, z)
     with pytest.raises(ValueError):
         w8a8.w8a8_dequant_per_tensor(Xq, s, z, out=torch.zeros((4, 32), dtype=torch.int32))
+
+
+def _decode_args(M=4, N=8, K=32):
+    """Well-formed CPU tensors for the Decode linear (shapes and dtypes only)."""
+    return dict(X=torch.zeros((M, K), dtype=torch.bfloat16), S=torch.ones(1), r=torch.ones(1),
+                Z=torch.zeros(1, dtype=torch.int32), Wq=torch.zeros((N, K), dtype=torch.int8),
+                s_w=torch.ones(N), colsum=torch.zeros(N, dtype=torch.int32), bias=torch.zeros(N))
+
+
+@pytest.mark.parametrize("fn", ["w8a8_linear_static", "w8a8_linear_static_noalloc"])
+@pytest.mark.parametrize("bad,what", [
+    (dict(out=torch.zeros((4, 7), dtype=torch.bfloat16)), "out"),       # out smaller than [M, N]
+    (dict(out=torch.zeros((4, 8), dtype=torch.float16)), "out"),        # dtype the C side has no code for
+    (dict(s_w=torch.ones(7)), "s_w"),                                   # shorter than N
+    (dict(colsum=torch.zeros(8, dtype=torch.int64)), "colsum"),
+    (dict(colsum=torch.zeros(7, dtype=torch.int32)), "colsum"),
+    (dict(bias=torch.zeros(7)), "bias"),
+    (dict(bias=torch.zeros(8, dtype=torch.float64)), "bias"),
+    (dict(X=torch.zeros((4, 32), dtype=torch.float32)), "X"),
+    (dict(X=torch.zeros((32, 4), dtype=torch.bfloat16).t()), "X"),     # rows not contiguous
+    (dict(Wq=torch.zeros((8, 16), dtype=torch.int8)), "Wq"),           # K differs from X's
+    (dict(Wq=torch.zeros((8, 32), dtype=torch.uint8)), "Wq"),
+    (dict(S=torch.ones(2)), "S"),
+    (dict(r=torch.ones(1, dtype=torch.float64)), "r"),
+    (dict(Z=torch.zeros(1, dtype=torch.int64)), "Z"),
+])
+def test_binding_rejects_bad_tensors_before_the_c_call(fn, bad, what):
+    """Every tensor the C side takes as a raw pointer of a fixed type and
+    extent is checked in the binding: a wrong shape or dtype raises
+    ValueError naming the argument, before anything is launched."""
+    a = _decode_args()
+    bad = dict(bad)
+    out = bad.pop("out", None)
+    a.update(bad)
+    with pytest.raises(ValueError, match=what):
+        getattr(w8a8, fn)(a["X"], a["S"], a["r"], a["Z"], a["Wq"], a["s_w"], a["colsum"], bias=a["bias"], out=out)
+
+
+def test_binding_rejects_host_tensors_and_bad_gemm_operands():
+    a = _decode_args()
+    with pytest.raises(ValueError, match="CUDA"):   # well-formed, but host memory
+        w8a8.w8a8_linear_static(a["X"], a["S"], a["r"], a["Z"], a["Wq"], a["s_w"], a["colsum"])
+    Xq = torch.zeros((4, 32), dtype=torch.int8)
+    with pytest.raises(ValueError, match="S_x"):
+        w8a8.w8a8_gemm_dequant(Xq, torch.ones(3), a["Wq"], a["s_w"])
+    with pytest.raises(ValueError, match="colsum"):
+        w8a8.w8a8_gemm_dequant(Xq, torch.ones(4), a["Wq"], a["s_w"], Z=a["Z"])
+    with pytest.raises(ValueError, match="out"):
+        w8a8.w8a8_gemm_dequant(Xq, torch.ones(4), a["Wq"], a["s_w"], out=torch.zeros((4, 8), dtype=torch.int8))
+    with pytest.raises(ValueError, match="W"):
+        w8a8.int8_mixed_decomp_gemm(Xq, torch.ones(4), torch.zeros((4, 16), dtype=torch.bfloat16),
+                                    torch.zeros(16, dtype=torch.int32), torch.zeros(1, dtype=torch.int32), 16,
+                                    a["Wq"], a["s_w"], torch.zeros((32, 7), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="Xo"):
+        w8a8.int8_outlier_split(a["X"], 6.0, 16, Xo=torch.zeros((4, 8), dtype=torch.bfloat16))
