@@ -265,11 +265,6 @@ __device__ __forceinline__ void quantize_stage(const uint8_t *xb, uint8_t *xq, i
   }
 }
 
-// Store a 32-bit word to a shared::cluster address (from map_to_rank).
-__device__ __forceinline__ void st_shared_cluster(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
 template <int MP, int SPLIT, bool FUSEQ>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     gemm_i8_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,

@@ -36,6 +36,7 @@
 // wait is bounded; on a timeout the CTA records W8A8_ERR_DEVICE_TIMEOUT,
 // stops, frees its TMEM and returns.
 #include "device.cuh"
+#include "gemm_pair.cuh"
 #include "kernels.h"
 
 namespace w8a8 {
@@ -579,8 +580,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *tempty_bar = tfull_bar + 2;
   uint64_t *cready_bar = tempty_bar + 2;  // a slot of sConst is written (one arrival per epilogue warp)
   uint64_t *drain_bar = cready_bar + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
+  uint64_t *exit_bar = drain_bar + 1;  // leader: rank 1's producer has published its fill count
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(exit_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *peer_fills = abort_flag + 1;  // leader: k-block loads rank 1 issued
+  volatile int *peer_abort = peer_fills + 1;  // leader: rank 1 gave up
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -600,7 +604,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&cready_bar[b], 4);  // one arrival per epilogue warp of this CTA
     }
     mbar_init(drain_bar, 1);
+    mbar_init(exit_bar, 1);
     *abort_flag = 0;
+    *peer_fills = 0;
+    *peer_abort = 0;
     fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -625,48 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer (both CTAs)
-      // The first ring of weight tiles does not depend on the previous kernel
-      // in the stream; the activation may, so its tiles follow the wait.
-      int pre = 0;
-      if (cluster_id < num_tiles) {
-        pre = nkb < STAGES ? nkb : STAGES;
-        const int32_t brow0 = static_cast<int32_t>((cluster_id / num_m) * kTileN + rank * kHalf);
-        for (int kb = 0; kb < pre; ++kb) {  // the ring starts empty: no waits
-          if (leader) mbar_arrive_expect_tx(&full_bar[kb], 2 * (kStageA2 + kStageB2));
-          tma_load_2d_pair(&tmB, map_to_rank(&full_bar[kb], 0), sB + kb * kStageB2, kb * kBK, brow0);
-        }
-      }
-      pdl_wait_prerequisite();
-      if (pre > 0) {
-        const int32_t arow0 = static_cast<int32_t>((cluster_id % num_m) * kTileM + rank * kHalf);
-        for (int kb = 0; kb < pre; ++kb)
-          tma_load_2d_pair(&tmA, map_to_rank(&full_bar[kb], 0), sA + kb * kStageA2, kb * kBK, arow0);
-      }
-      int stage = pre % STAGES;
-      uint32_t phase = pre == STAGES ? 1u : 0u;
-      bool ok = true;
-      for (int64_t tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
-        const int32_t arow = static_cast<int32_t>((tile % num_m) * kTileM + rank * kHalf);
-        const int32_t brow = static_cast<int32_t>((tile / num_m) * kTileN + rank * kHalf);
-        for (int kb = tile == cluster_id ? pre : 0; kb < nkb; ++kb) {
-          if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag, limit_ns)) {
-            ok = false;
-            break;
-          }
-          const uint32_t leader_full = map_to_rank(&full_bar[stage], 0);
-          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * (kStageA2 + kStageB2));
-          tma_load_2d_pair(&tmA, leader_full, sA + stage * kStageA2, kb * kBK, arow);
-          tma_load_2d_pair(&tmB, leader_full, sB + stage * kStageB2, kb * kBK, brow);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (!ok) {
-        record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
-        *abort_flag = 1;
-      }
+      pair_tma_producer<STAGES>(&tmA, &tmB, sA, sB, full_bar, empty_bar, PairExitWords{exit_bar, peer_fills, peer_abort},
+                                abort_flag, num_m, num_tiles, nkb, cluster_id, num_clusters, rank, status, limit_ns);
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -821,7 +788,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int STAGES, bool MIXED>
 cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                          const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
+  // ring + epilogue constants + 1 KiB alignment slack + barriers and flags (< 256 B)
   constexpr size_t kSmem = static_cast<size_t>(STAGES) * 2 * 128 * kBK + 2 * 3 * 256 * 4 + 1024 + 256;
+  static_assert((2 * STAGES + 7) * 8 + 4 * 4 <= 256, "barriers and flags fit their reserve");
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   alignas(64) CUtensorMap tmA, tmB;
   if (!encode_tmap_2d(&tmA, Xq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
