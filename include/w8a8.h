@@ -279,24 +279,25 @@ w8a8_status w8a8_gemm_requant(const int8_t *Xq, const float *S_x, int32_t s_x_pe
 /*
  * w8a8_linear_static without a workspace argument: the same computation and
  * result as w8a8_linear_static (same arguments, same checks), for callers
- * that cannot allocate device memory when they run a Decode step -- a CUDA
- * graph being captured (cudaMalloc is not a stream operation and breaks the
- * capture), a plug-in inside a runtime that owns all device memory, or a
- * latency-critical step that cannot take an allocation's implicit device
- * synchronization. No counterpart on the pages: this is a deployment entry
- * point of this library.
+ * that cannot allocate device memory when they run a Decode step -- a
+ * plug-in inside a runtime that owns every byte of device memory and hands
+ * none out, or a latency-critical step that cannot take the device-wide
+ * synchronization a cudaMalloc / cudaFree may cause. No counterpart on the
+ * pages: this is a deployment entry point of this library.
  * It always computes in two kernels -- the static quantization into a
  * scratch, then the Decode-shaped GEMM -- where w8a8_linear_static fuses both
- * for some shapes; the results are identical. The scratch (the quantized activation) is one fixed device
- * array inside the library, 524,288 bytes (32 tokens x 16384), held by every
- * GPU that loads the library until the process exits. It serves M <= 32,
- * N <= 32768 and K <= 16384; larger shapes return W8A8_ERR_UNSUPPORTED_SHAPE
- * without launching anything. The call allocates nothing.
+ * for some shapes; the results are identical. The scratch (the quantized
+ * activation) is one fixed device array inside the library, 524,288 bytes
+ * (32 tokens x 16384), held by every GPU that loads the library until the
+ * process exits. It serves M <= 32, N <= 32768 and K <= 16384; larger shapes
+ * return W8A8_ERR_UNSUPPORTED_SHAPE without launching anything. The call
+ * allocates nothing (no cudaMalloc, no allocating library routine).
  * The first call on a device also sets up that device (looks up the array's
- * device address and zero-fills it once, synchronously): make that first
- * call before any stream capture. All calls on a device share the one array,
- * which keeps the last call's contents, so calls that overlap on the GPU
- * (different streams, or concurrent graphs) race: serialize them.
+ * device address with cudaGetSymbolAddress and zero-fills it once,
+ * synchronously): make that first call before any stream capture. All calls
+ * on a device share the one array, which keeps the last call's contents
+ * (every byte a call reads is written earlier by the same call), so calls
+ * that overlap on the GPU (different streams) race: serialize them.
  */
 w8a8_status w8a8_linear_static_noalloc(const void *X, int64_t M, int64_t K, int64_t ldx, const float *S,
                                        const float *r, const int32_t *Z, const int8_t *Wq,
@@ -356,6 +357,32 @@ w8a8_status int8_mixed_decomp_gemm(const int8_t *Xq, const float *S_x, const voi
                                    const int8_t *Wq, const float *s_w, const void *W, int64_t ldw,
                                    const float *bias, int64_t M, int64_t N, int64_t K, void *out,
                                    w8a8_dtype out_dtype, void *stream);
+
+/*
+ * int8_mixed_decomp_gemm with the 16-bit side product on the tensor cores:
+ * the same arguments, checks and formula, except that
+ *   side[m, n] = sum_{j < n_used} Xo[m, j] * W[idx[j], n]
+ * is formed by bf16 x bf16 -> fp32 tensor-core MMAs (tcgen05.mma kind::f16)
+ * in the hardware's summation order instead of the ascending fmaf chain.
+ * The products are exact in fp32, so side differs from the chain only by
+ * fp32 rounding of the sum: |side - side_chain| <= 2 n_used 2^-23
+ * sum_j |Xo[m, j] W[idx[j], n]|; y then follows the same fixed-order epilogue
+ * (y = fmaf((float) acc, S_x[m] * s_w[n], side + bias[n])). Built for heavy
+ * outlier loads: its cost grows with ceil(n_used / 64) MMA k-blocks on the
+ * tensor pipe rather than with n_used fmaf per output element.
+ * Source: LLM.int8() summary, 16-bit decomposition step (2) (X_F16 W_F16 for
+ * the outlier columns, then summed with the dequantized INT8 product) and
+ * the mixed-precision decomposition formula Y. Reading: the pages' FP16 side
+ * GEMM is taken as bf16 inputs with fp32 accumulation, as in
+ * int8_mixed_decomp_gemm.
+ * Any M; Xo and W 16-byte aligned; the columns of Xo at or past n_used are
+ * not read.
+ */
+w8a8_status int8_mixed_decomp_gemm_tc(const int8_t *Xq, const float *S_x, const void *Xo,
+                                      const int32_t *outlier_idx, const int32_t *n_out, int32_t cap,
+                                      const int8_t *Wq, const float *s_w, const void *W, int64_t ldw,
+                                      const float *bias, int64_t M, int64_t N, int64_t K, void *out,
+                                      w8a8_dtype out_dtype, void *stream);
 
 /*
  * Device status word. Kernels record device-side failures (a bounded wait

@@ -195,7 +195,7 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
   DeviceInfo *d;
   if (w8a8_status s = device_info(&d)) return s;
   return from_cuda(launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq,
-                                           d->sm_count, static_cast<cudaStream_t>(stream)));
+                                           d->sm_count, static_cast<cudaStream_t>(stream), /*pdl=*/true));
 }
 
 w8a8_status w8a8_dequant_per_tensor(const int8_t *Xq, int64_t M, int64_t K, int64_t ldq, const float *S,
@@ -403,6 +403,51 @@ w8a8_status int8_outlier_split(const void *X, int64_t M, int64_t K, int64_t ldx,
   return from_cuda(launch_outlier_split(static_cast<const uint16_t *>(X), M, K, ldx, threshold, cap, Xq, S_x,
                                         outlier_idx, n_out, static_cast<uint16_t *>(Xo), workspace, d->sm_count,
                                         d->status, static_cast<cudaStream_t>(stream)));
+}
+
+// Shared by int8_mixed_decomp_gemm and int8_mixed_decomp_gemm_tc: checks and
+// the epilogue operands.
+static w8a8_status check_mixed(const int8_t *Xq, const float *S_x, const void *Xo, const int32_t *outlier_idx,
+                               const int32_t *n_out, int32_t cap, const int8_t *Wq, const float *s_w, const void *W,
+                               int64_t ldw, const float *bias, int64_t M, int64_t N, int64_t K, void *out,
+                               w8a8_dtype out_dtype, EpilogueArgs *ep) {
+  if (w8a8_status s = check_gemm_common(Xq, Wq, s_w, bias, nullptr, M, N, K, out, out_dtype)) return s;
+  if (out_dtype == W8A8_I32) return W8A8_ERR_UNSUPPORTED_DTYPE;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if (!S_x || !n_out || cap < 0 || cap > 4096 || (cap > 0 && (!Xo || !outlier_idx || !W)) ||
+      ldw < N)
+    return W8A8_ERR_INVALID_ARG;
+  if ((Xo && !aligned16(Xo)) || (W && !aligned16(W))) return W8A8_ERR_MISALIGNED;
+  ep->S_x = S_x;
+  ep->s_x_per_row = 1;
+  ep->s_w = s_w;
+  ep->bias = bias;
+  ep->Xo = static_cast<const uint16_t *>(Xo);
+  ep->outlier_idx = outlier_idx;
+  ep->n_out = n_out;
+  ep->cap = cap;
+  ep->W = static_cast<const uint16_t *>(W);
+  ep->ldw = ldw;
+  ep->out = out;
+  ep->out_dtype = out_dtype;
+  return W8A8_OK;
+}
+
+w8a8_status int8_mixed_decomp_gemm_tc(const int8_t *Xq, const float *S_x, const void *Xo,
+                                      const int32_t *outlier_idx, const int32_t *n_out, int32_t cap,
+                                      const int8_t *Wq, const float *s_w, const void *W, int64_t ldw,
+                                      const float *bias, int64_t M, int64_t N, int64_t K, void *out,
+                                      w8a8_dtype out_dtype, void *stream) {
+  EpilogueArgs ep;
+  if (w8a8_status s = check_mixed(Xq, S_x, Xo, outlier_idx, n_out, cap, Wq, s_w, W, ldw, bias, M, N, K, out,
+                                  out_dtype, &ep))
+    return s;
+  if (M == 0 || N == 0) return W8A8_OK;
+  DeviceInfo *d;
+  if (w8a8_status s = device_info(&d)) return s;
+  if (d->sm_count < 2) return W8A8_ERR_NO_DEVICE;
+  return from_cuda(launch_gemm_side_tc(Xq, Wq, M, N, K, ep, d->sm_count, d->status,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 w8a8_status int8_mixed_decomp_gemm(const int8_t *Xq, const float *S_x, const void *Xo,

@@ -81,6 +81,11 @@ cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_
                            const EpilogueArgs &ep, bool mixed, int num_sms, int32_t *status,
                            cudaStream_t s);
 
+// LLM.int8() mixed GEMM with the 16-bit side product on the tensor cores
+// (CTA pairs, one int32 and one fp32 TMEM accumulator per tile; any M).
+cudaError_t launch_gemm_side_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
+                                const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s);
+
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_t s);
 
 // Decode-shaped GEMM (M <= 64): one cluster of decode_split(M, N, K) CTAs

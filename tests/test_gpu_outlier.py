@@ -21,9 +21,14 @@ def assert_same(gpu, ref, what):
     assert eq.all(), f"{what}: " + diff_report(gpu, ref)
 
 
-def planted(M, K, cols, seed, lo=20.0, hi=100.0):
+def planted(M, K, cols, seed, lo=20.0, hi=100.0, clip=None):
+    """N(0,1) [M, K] (optionally clipped to +-clip, so that only the planted
+    columns can exceed a threshold above it) with `cols` replaced by random
+    sign x U(lo, hi)."""
     rng = np.random.default_rng(seed)
     x = rng.standard_normal((M, K)).astype(np.float32)
+    if clip is not None:
+        x = np.clip(x, -clip, clip)
     mag = rng.uniform(lo, hi, size=(M, len(cols))).astype(np.float32)
     sign = np.where(rng.random((M, len(cols))) < 0.5, -1.0, 1.0).astype(np.float32)
     x[:, cols] = sign * mag
@@ -95,10 +100,11 @@ def test_mixed_decomp_gemm_bit_exact(M, K, N, cols, out_dtype):
     assert W.w8a8_check_device_error() == 0
 
 
-def test_llm_int8_full_size_sampled():
+def test_llm_int8_full_size():
     """X [4096, 8192] with 6-8 planted outlier columns, W bf16 [8192, 8192]:
-    the split is compared in full, the output on 96 x 96 sampled elements
-    computed one by one by the oracle."""
+    the split and every element of the mixed GEMM's output compared with the
+    oracle (the INT8 product, the 16-bit side product and the epilogue over
+    the whole layer)."""
     case = synth.llm_int8(0)
     cap = 64
     Wd = dev_bf16(case.W)
@@ -112,13 +118,95 @@ def test_llm_int8_full_size_sampled():
     assert_same(host(Xq), rq, "Xq")
     assert_same(host(S_x), rS, "S_x")
     assert_same(host_bf16(Xo)[:, :rn], rXo[:, :rn], "Xo")
-    rng = np.random.default_rng(7)
-    rows = np.sort(rng.choice(4096, 96, replace=False))
-    cols = np.sort(rng.choice(8192, 96, replace=False))
-    Wsub = np.ascontiguousarray(case.W[:, cols])
-    rwq, rws, _ = oracle.quant_weight_per_channel(Wsub)   # per-channel: columns are independent
-    acc = oracle.gemm_i64(rq[rows], rwq)
-    side = oracle.outlier_side(rXo[rows], ridx, Wsub)
-    y = oracle.epilogue(acc, rS[rows], rws, side=side)
-    assert_same(host_bf16(out)[np.ix_(rows, cols)], oracle.f32_to_bf16(y), "sampled out")
+    rwq, rws, _ = oracle.quant_weight_per_channel(case.W)
+    assert_same(host(Wq), rwq, "Wq")
+    assert_same(host(s_w), rws, "s_w")
+    side = oracle.outlier_side(rXo, ridx, case.W)
+    y = oracle.epilogue(oracle.gemm_i64(rq, rwq), rS, rws, side=side)
+    assert_same(host_bf16(out), oracle.f32_to_bf16(y), "out")
     assert W.w8a8_check_device_error() == 0
+
+
+# ------------------------------------------------------------ tensor-core side product
+U = 2.0 ** -23  # one fp32 ulp at 1.0 (an upper bound on the unit roundoff under any rounding rule)
+
+
+def side_tolerance(Xo_bits, idx, W_bits, side_ref, bias, y_ref):
+    """Per-element bound on |y_tc - y_oracle| when only the summation order of
+    the side product differs. The products Xo[m, j] W[idx[j], n] are exact
+    in fp32, and any order of n additions in fp32 is within
+    (n - 1) u sum_j |products| of the exact sum, so two orders differ by at
+    most 2 n u S_abs (S_abs = sum_j |product|, in float64 here). The
+    epilogue then rounds side + bias once and the fma once, which moves y by
+    at most one ulp of each of those results more."""
+    n = len(idx)
+    xo = np.abs(oracle.bf16_to_f32(Xo_bits[:, :n]).astype(np.float64))
+    w = np.abs(oracle.bf16_to_f32(W_bits[idx]).astype(np.float64))
+    s_abs = xo @ w
+    b = 0.0 if bias is None else np.abs(bias.astype(np.float64))[None, :]
+    return U * (2 * n * s_abs + np.abs(side_ref) + b + 2 * np.abs(y_ref)) + 1e-30, s_abs
+
+
+@pytest.mark.parametrize("M,K,N,n_cols,cap,with_bias", [
+    (300, 1024, 520, 0, 16, True),      # no outlier: the side accumulator is never read
+    (300, 1024, 520, 8, 8, True),       # one side k-block, mostly padding
+    (129, 2048, 1000, 64, 64, False),   # exactly one full side k-block
+    (520, 2048, 777, 65, 70, True),     # two k-blocks, Xo rows not 16-byte multiples (cap 70)
+    (512, 2048, 1024, 512, 512, True),  # eight k-blocks through the double-buffered side ring
+    (256, 8192, 512, 4096, 4096, False),  # the largest cap
+    (16, 512, 300, 40, 48, True),       # fewer tokens than one pair tile
+])
+def test_mixed_decomp_gemm_tc_within_derived_bound(M, K, N, n_cols, cap, with_bias):
+    rng = np.random.default_rng(M + K + n_cols)
+    cols = np.sort(rng.choice(K, n_cols, replace=False)) if n_cols else np.array([], np.int64)
+    X = planted(M, K, cols.tolist(), seed=7 * M + n_cols, clip=5.5)  # exactly the planted columns exceed 6
+    Wb = synth.bf16_bits(synth.weight(np.random.default_rng(N + n_cols), K, N))
+    bias = synth.bias(np.random.default_rng(9), N) if with_bias else None
+    Wd = dev_bf16(Wb)
+    Wq, s_w, _ = W.w8a8_quant_weight_per_channel(Wd)
+    Xq, S_x, idx, n_out, Xo = W.int8_outlier_split(dev_bf16(X), 6.0, cap)
+    b = None if bias is None else dev(bias)
+    y32 = W.int8_mixed_decomp_gemm_tc(Xq, S_x, Xo, idx, n_out, cap, Wq, s_w, Wd, bias=b, out_dtype=torch.float32)
+    y16 = W.int8_mixed_decomp_gemm_tc(Xq, S_x, Xo, idx, n_out, cap, Wq, s_w, Wd, bias=b)
+    assert W.w8a8_check_device_error() == 0
+    rq, rS, ridx, rn, rXo = oracle.outlier_split(X, 6.0, cap)
+    assert rn == n_cols and int(host(n_out)[0]) == rn
+    rwq, rws, _ = oracle.quant_weight_per_channel(Wb)
+    side = oracle.outlier_side(rXo, ridx, Wb)
+    y_ref = oracle.epilogue(oracle.gemm_i64(rq, rwq), rS, rws, bias=bias, side=side)
+    got = host(y32)
+    # the bf16 result is the fp32 result rounded once (same kernel, same order)
+    assert_same(host_bf16(y16), oracle.f32_to_bf16(got), "bf16 out vs the fp32 out rounded")
+    if n_cols == 0:  # no side product at all: the fixed-order epilogue, bit for bit
+        assert_same(got, y_ref, "out")
+        return
+    tol, s_abs = side_tolerance(rXo, ridx, Wb, side, bias, y_ref)
+    err = np.abs(got.astype(np.float64) - y_ref.astype(np.float64))
+    bad = np.argwhere(err > tol)
+    assert bad.size == 0, f"{len(bad)} elements outside the bound; first {bad[:3].tolist()}: " \
+                          f"{[(got[tuple(i)], y_ref[tuple(i)], tol[tuple(i)]) for i in bad[:3]]}"
+    # the target's 1e-3 relative error per element, wherever the side sum is
+    # well conditioned (2 n u S_abs <= 1e-4 |y|); near cancellation no fp32
+    # summation order, the oracle's included, is that close to the exact sum
+    wc = 2 * n_cols * U * s_abs <= 1e-4 * np.abs(y_ref)
+    assert (err[wc] <= 1e-3 * np.abs(y_ref[wc])).all()
+
+
+def test_llm_int8_full_size_tensor_core_side():
+    """The LLM.int8() workload (4096 x 8192 -> 8192, 6-8 outlier columns)
+    through the tensor-core side product: every output element within the
+    derived bound of the oracle."""
+    case = synth.llm_int8(0)
+    cap = 64
+    Wd = dev_bf16(case.W)
+    Wq, s_w, _ = W.w8a8_quant_weight_per_channel(Wd)
+    Xq, S_x, idx, n_out, Xo = W.int8_outlier_split(dev_bf16(case.X), case.threshold, cap)
+    y32 = W.int8_mixed_decomp_gemm_tc(Xq, S_x, Xo, idx, n_out, cap, Wq, s_w, Wd, out_dtype=torch.float32)
+    assert W.w8a8_check_device_error() == 0
+    rq, rS, ridx, rn, rXo = oracle.outlier_split(case.X, case.threshold, cap)
+    rwq, rws, _ = oracle.quant_weight_per_channel(case.W)
+    side = oracle.outlier_side(rXo, ridx, case.W)
+    y_ref = oracle.epilogue(oracle.gemm_i64(rq, rwq), rS, rws, side=side)
+    tol, _ = side_tolerance(rXo, ridx, case.W, side, None, y_ref)
+    err = np.abs(host(y32).astype(np.float64) - y_ref.astype(np.float64))
+    assert (err <= tol).all(), f"{int((err > tol).sum())} elements outside the bound"
