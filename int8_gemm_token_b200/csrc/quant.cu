@@ -41,9 +41,11 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__
   const uint16_t *xrow = X + m * ldx;
   // Launched with programmatic stream serialization, this kernel may start
   // while the previous kernel still runs: let the dependent GEMM launch (it
-  // touches nothing this kernel writes before its own wait), then wait for the
-  // previous kernel before reading X or writing Xq, S_x.
+  // touches nothing this kernel writes before its own wait), ask L2 for this
+  // block's rows, then wait for the previous kernel before reading X or
+  // writing Xq, S_x.
   pdl_launch_dependents();
+  if (t == 0 && row_ok) prefetch_l2_bulk(xrow, static_cast<uint32_t>(K * 2));
   pdl_wait_prerequisite();
 
   uint4 v[VPT];
@@ -124,11 +126,18 @@ __global__ void __launch_bounds__(256) quant_per_tensor_kernel(const uint16_t *_
   // which returns after this kernel has completed), then waits for the
   // previous kernel before reading X or writing Xq.
   pdl_launch_dependents();
+  const int64_t cpr = K >> 3;  // chunks per row
+  const int64_t total = M * cpr;
+  // dense rows: the first 4 KiB span of X this block converts, asked of L2
+  // before the wait (only the first: asking for more than the block consumes
+  // right away lets later spans evict earlier ones)
+  if (ldx == K && threadIdx.x * 32 < blockDim.x) {
+    const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x * 32;
+    if (i < total) prefetch_l2_bulk(X + i * 8, static_cast<uint32_t>((total - i < 32 ? total - i : 32) * 16));
+  }
   pdl_wait_prerequisite();
   const float r = *r_ptr;
   const int z = *Z_ptr;
-  const int64_t cpr = K >> 3;  // chunks per row
-  const int64_t total = M * cpr;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t m = i / cpr, c = i - m * cpr;
@@ -166,10 +175,19 @@ __global__ void __launch_bounds__(256) dequant_per_tensor_kernel(const int8_t *_
                                                                  const float *__restrict__ S_ptr,
                                                                  const int32_t *__restrict__ Z_ptr,
                                                                  void *__restrict__ out) {
-  const float S = *S_ptr;
-  const int z = *Z_ptr;
+  // Programmatic dependent launch: let the next kernel launch, ask L2 for
+  // this block's codes (dense rows), then wait for the previous kernel before
+  // reading Xq, S, Z or writing `out`.
+  pdl_launch_dependents();
   const int64_t cpr = K >> 4;  // 16-code chunks per row
   const int64_t total = M * cpr;
+  if (ldq == K && threadIdx.x * 32 < blockDim.x) {  // the block's first span, as in quant_per_tensor
+    const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x * 32;
+    if (i < total) prefetch_l2_bulk(Xq + i * 16, static_cast<uint32_t>((total - i < 32 ? total - i : 32) * 16));
+  }
+  pdl_wait_prerequisite();
+  const float S = *S_ptr;
+  const int z = *Z_ptr;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t m = i / cpr, c = i - m * cpr;
@@ -201,12 +219,17 @@ cudaError_t launch_dequant_per_tensor(const int8_t *Xq, int64_t M, int64_t K, in
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
-  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
-  if (bf16_out)
-    dequant_per_tensor_kernel<true><<<grid, block, 0, s>>>(Xq, M, K, ldq, S, Z, out);
-  else
-    dequant_per_tensor_kernel<false><<<grid, block, 0, s>>>(Xq, M, K, ldq, S, Z, out);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (bf16_out) return cudaLaunchKernelEx(&cfg, dequant_per_tensor_kernel<true>, Xq, M, K, ldq, S, Z, out);
+  return cudaLaunchKernelEx(&cfg, dequant_per_tensor_kernel<false>, Xq, M, K, ldq, S, Z, out);
 }
 
 // ------------------------------------------------------------ calibration
