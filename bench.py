@@ -118,7 +118,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.005)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self.nv is not None:
@@ -264,22 +264,24 @@ def run_ours(args, world, rank, local):
     # The steps run back to back with events only at both ends: the kernels
     # use programmatic dependent launch, so each one starts under the tail of
     # the one before, and an event recorded between two kernels would stop that.
+    # The clock sampler runs over this region and the per-kernel passes below.
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(sets[i % N_SETS])
-        t1.record(stream)
-        torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.__enter__()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(sets[i % N_SETS])
+    t1.record(stream)
+    torch.cuda.synchronize()
     barrier()
     total_ms = t0.elapsed_time(t1)
     ms_per_step = max_ranks(total_ms / args.steps)
-    # Per-kernel durations (roofline, quant row): a second timed pass with
-    # events around each kernel, which serialises them.
-    n_bd = max(3, min(args.steps, 200))
+    # Per-kernel durations (burst roofline, quant row): a second pass of 200
+    # steps with events around each kernel, which serialises them.
+    n_bd = 200
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_bd)]
     torch.cuda.synchronize()
     for i in range(n_bd):
@@ -292,41 +294,97 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     quant_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     gemm_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    # Sustained: the GEMM alone, back to back for >= 1 s (the power cap sets
+    # the clock there), events only at both ends.
+    gemm = lambda s: W.w8a8_gemm_dequant(s["Xq"], s["S"], s["Wq"], s["s_w"], bias=s["bias"], out=s["out"],
+                                         stream=stream)
+    n_sus, sus_ms = 0, 0.0
+    while sus_ms < 1000.0 and not args.no_sustained:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(2000):
+            gemm(sets[i % N_SETS])
+        b.record(stream)
+        torch.cuda.synchronize()
+        sus_ms += a.elapsed_time(b)
+        n_sus += 2000
+    clocks.__exit__()
     ops = 2.0 * M * N * K
     value = whole_job_tops(ops, world, ms_per_step)
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
+    sus_tops = ops * n_sus / (sus_ms * 1e-3) / 1e12 if n_sus else None
     quant_bytes = 2.0 * M * K + M * K + 4.0 * M
     quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
     if W.w8a8_check_device_error() != 0:
         raise RuntimeError("device status word set during the benchmark")
+    c1 = None if args.no_c1 else bench_c1(dev)
 
     # ---------------------------------------------------------------- e2e
+    # The same step through the public API from and to pinned host memory:
+    # each step copies its X in (host -> device) and its bf16 output back
+    # (device -> host). Three streams with two device buffer sets let the
+    # input copy of step i+1 and the output copy of step i-1 run while step i
+    # computes (PCIe is full duplex); events order every buffer's reuse.
     e2e = None
     if not args.no_e2e:
+        e2e_steps = max(2 * N_SETS, min(args.steps, 50))
+        nb = 2
         hostX = [sets[i]["X"].cpu().pin_memory() for i in range(N_SETS)]
         hostOut = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(N_SETS)]
-        e2e_steps = max(3, min(args.steps, 50))
-        for i in range(3):
-            s = sets[i % N_SETS]
-            s["X"].copy_(hostX[i % N_SETS], non_blocking=True)
-            step(s)
-            hostOut[i % N_SETS].copy_(s["out"], non_blocking=True)
+        # one layer (the weight of set 0) serves every step, as in a serving loop
+        bufs = [dict(sets[0], X=torch.empty_like(sets[0]["X"]), out=torch.empty_like(sets[0]["out"]))
+                for _ in range(nb)]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+        def e2e_run(n):
+            copied_in = [None] * nb    # X[b] holds step i's input
+            computed = [None] * nb     # out[b] holds step i's output
+            drained = [None] * nb      # out[b] has been copied to the host
+            used = [None] * nb         # step i's kernels have read X[b]
+            for i in range(n):
+                b = i % nb
+                with torch.cuda.stream(s_in):
+                    if used[b] is not None:
+                        s_in.wait_event(used[b])
+                    bufs[b]["X"].copy_(hostX[i % N_SETS], non_blocking=True)
+                    copied_in[b] = torch.cuda.Event()
+                    copied_in[b].record(s_in)
+                stream.wait_event(copied_in[b])
+                if drained[b] is not None:
+                    stream.wait_event(drained[b])
+                step(bufs[b])
+                used[b] = computed[b] = torch.cuda.Event()
+                computed[b].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(computed[b])
+                    hostOut[i % N_SETS].copy_(bufs[b]["out"], non_blocking=True)
+                    drained[b] = torch.cuda.Event()
+                    drained[b].record(s_out)
+            for ev_ in drained:
+                if ev_ is not None:
+                    stream.wait_event(ev_)
+
+        e2e_run(3)
         torch.cuda.synchronize()
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(e2e_steps):
-            s = sets[i % N_SETS]
-            s["X"].copy_(hostX[i % N_SETS], non_blocking=True)
-            step(s)
-            hostOut[i % N_SETS].copy_(s["out"], non_blocking=True)
+        e2e_run(e2e_steps)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_ranks(e0.elapsed_time(e1) / e2e_steps)
+        ok = True
+        for j in range(N_SETS):  # the last step that used input j, recomputed on the device
+            ref = dict(bufs[0], X=sets[j]["X"], out=torch.empty_like(bufs[0]["out"]))
+            step(ref)
+            ok = ok and torch.equal(hostOut[j], ref["out"].cpu())
         e2e = {"value": whole_job_tops(ops, world, e2e_ms), "unit": "TOPS",
                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms,
-               "steps": e2e_steps}
+               "steps": e2e_steps, "outputs_match_device_run": ok,
+               "timing": "pinned host X -> device, quant + GEMM, bf16 out -> pinned host, every step; input, "
+                         "compute and output copies on three streams with two device buffer sets"}
+        del bufs
 
     del sets
     torch.cuda.empty_cache()
@@ -356,18 +414,25 @@ def run_ours(args, world, rank, local):
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": workload_config(world),
             "roofline": {"bound": "tensor", "kernel": "gemm_i8_tc2_kernel", "achieved": gemm_tops,
-                         "peak": int8_sustained, "unit": "TOPS", "frac": gemm_tops / int8_sustained,
-                         "peak_source": f"{peaks['source']} sustained bf16 {peaks['bf16_tflops_sustained']} TFLOP/s x 2 "
-                                        "(int8/bf16 nominal); the kernel is timed right after the K-step loop",
-                         "frac_of_burst_peak": gemm_tops / int8_peak,
+                         "peak": int8_peak, "unit": "TOPS", "frac": gemm_tops / int8_peak,
+                         "peak_source": f"{peaks['source']} burst bf16 {peaks['bf16_tflops']} TFLOP/s x 2 "
+                                        "(int8/bf16 nominal ratio); the kernel is timed in 200 launches with "
+                                        "events around each",
                          "traffic": profiled_traffic(TC2_TRAFFIC), "traffic_unit": "B per launch",
                          "traffic_profile": TC2_TRAFFIC["profile"],
-                         "algorithmic_bytes": M * K + N * K + 2 * M * N + 4 * M + 8 * N},
+                         "algorithmic_ops": ops,
+                         "algorithmic_bytes": M * K + N * K + 2 * M * N + 4 * M + 8 * N,
+                         "sustained": None if sus_tops is None else {
+                             "achieved": sus_tops, "peak": int8_sustained, "frac": sus_tops / int8_sustained,
+                             "launches": n_sus, "ms": sus_ms,
+                             "peak_source": f"{peaks['source']} sustained bf16 {peaks['bf16_tflops_sustained']} "
+                                            "TFLOP/s x 2; the GEMM alone back to back for >= 1 s"}},
             "quant": {"kernel": "quant_per_token_kernel", "ms": quant_ms, "achieved": quant_gbs,
                       "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": quant_gbs / peaks["hbm_gbs"],
                       "C_s_over_C_g": quant_ms / gemm_ms, "timing": "events around each launch in the step",
                       "stream": quant_stream},
             "gemm_ms": gemm_ms,
+            "prefill_small": c1,
             "decode": decode,
             "kv_cache": kv,
             "llm_int8": llm,
@@ -378,7 +443,9 @@ def run_ours(args, world, rank, local):
             "timing": {"value": "K back-to-back steps between two CUDA events (kernels overlap through "
                                 "programmatic dependent launch)",
                        "per_kernel": f"{n_bd} further steps with events around each kernel (serialised); "
-                                     "roofline.achieved and quant use these"},
+                                     "roofline.achieved and quant use these",
+                       "clocks": "NVML samples every 2 ms over the timed steps, the per-kernel pass and the "
+                                 ">= 1 s sustained GEMM pass"},
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -410,6 +477,41 @@ def graph_time_us(fn, n_calls, reps=10):
     torch.cuda.synchronize()
     del g
     return a.elapsed_time(b) * 1e3 / (reps * n_calls)
+
+
+def bench_c1(dev):
+    """The small single-linear Prefill workload (16 tokens x 256 -> 512, seed
+    0): per-token quantization + GEMM + dequant, launch-latency bound. Per
+    call: back to back in a CUDA graph, and one call with events around it."""
+    import torch
+
+    from int8_gemm_token_b200 import synth
+    from int8_gemm_token_b200 import w8a8 as W
+    case = synth.prefill_small(0)
+    X = torch.from_numpy(case.X.view(np.int16)).view(torch.bfloat16).to(dev)
+    Wq, s_w, _ = W.w8a8_quant_weight_per_channel(torch.from_numpy(case.W).to(dev))
+    bias = torch.from_numpy(case.bias).to(dev)
+    Xq = torch.empty((16, 256), dtype=torch.int8, device=dev)
+    S = torch.empty((16,), dtype=torch.float32, device=dev)
+    out = torch.empty((16, 512), dtype=torch.bfloat16, device=dev)
+
+    def call(i):
+        W.w8a8_quant_per_token(X, Xq=Xq, S_x=S)
+        W.w8a8_gemm_dequant(Xq, S, Wq, s_w, bias=bias, out=out)
+    graph_us = graph_time_us(call, 20)
+    single = []
+    for _ in range(50):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        call(0)
+        b.record()
+        torch.cuda.synchronize()
+        single.append(a.elapsed_time(b) * 1e3)
+    return {"workload": "prefill single linear: X bf16 [16 x 256] row-scaled N(0,1) -> per-token quant -> INT8 "
+                        "GEMM vs W [256 x 512] + bias -> bf16 [16 x 512]",
+            "us_per_linear_graph": graph_us, "us_per_linear_single_call_median": statistics.median(single),
+            "ops": 2.0 * 16 * 256 * 512, "bound": "launch latency (4.2 MOP, 8 KB of activation)"}
 
 
 def bench_quant_stream(dev, peaks):
@@ -533,7 +635,10 @@ def bench_decode(args, dev, rank, peaks):
 
 
 def bench_llm_int8(args, dev, rank, peaks, int8_peak):
-    """LLM.int8() mode at 4096 x 8192 x 8192: outlier split + mixed GEMM."""
+    """LLM.int8() mode at 4096 x 8192 x 8192: the outlier split, and the mixed
+    GEMM with the side product on CUDA cores (fixed-order fmaf chain) and on
+    the tensor cores, at the workload's own 6-8 outlier columns and with 64
+    and 512 planted ones; the plain pair GEMM of the same shape for scale."""
     import torch
 
     from int8_gemm_token_b200 import synth
@@ -543,28 +648,57 @@ def bench_llm_int8(args, dev, rank, peaks, int8_peak):
     X, Wd = bf(case.X), bf(case.W)
     Mq, Kq = case.X.shape
     Nq = case.W.shape[1]
-    cap = 64
+    ops = 2.0 * Mq * Nq * Kq
     Wq, s_w, _ = W.w8a8_quant_weight_per_channel(Wd)
     Xq = torch.empty((Mq, Kq), dtype=torch.int8, device=dev)
     S = torch.empty((Mq,), dtype=torch.float32, device=dev)
-    idx = torch.empty((cap,), dtype=torch.int32, device=dev)
-    n_out = torch.empty((1,), dtype=torch.int32, device=dev)
-    Xo = torch.empty((Mq, cap), dtype=torch.bfloat16, device=dev)
     out = torch.empty((Mq, Nq), dtype=torch.bfloat16, device=dev)
     wsb = torch.zeros((W.lib().int8_outlier_split_workspace_size(Kq),), dtype=torch.uint8, device=dev)
-    split = lambda i: W.int8_outlier_split(X, case.threshold, cap, Xq=Xq, S_x=S, idx=idx, n_out=n_out, Xo=Xo, workspace=wsb)
-    gemm = lambda i: W.int8_mixed_decomp_gemm(Xq, S, Xo, idx, n_out, cap, Wq, s_w, Wd, out=out)
-    split_us = graph_time_us(split, 4)
-    gemm_us = graph_time_us(gemm, 4)
-    split_bytes = 2.0 * Mq * Kq + Mq * Kq + 4.0 * Mq + 2.0 * Mq * int(n_out.item())
-    ops = 2.0 * Mq * Nq * Kq
+    res = {"workload": f"LLM.int8() X [{Mq} x {Kq}], W bf16 [{Kq} x {Nq}], threshold 6.0", "rows": []}
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    for label in ("workload", 64, 512):
+        if label == "workload":
+            Xl, cap = X, 64
+        else:  # N(0,1) clipped to +-5.5 with `label` planted columns of random sign x U(20, 100)
+            cap = label
+            Xl = torch.randn((Mq, Kq), device=dev, generator=g).clamp_(-5.5, 5.5)  # only planted columns exceed 6
+            cols = torch.randperm(Kq, device=dev, generator=g)[:label]
+            mag = 20.0 + 80.0 * torch.rand((Mq, label), device=dev, generator=g)
+            sign = torch.where(torch.rand((Mq, label), device=dev, generator=g) < 0.5, -1.0, 1.0)
+            Xl[:, cols] = sign * mag
+            Xl = Xl.to(torch.bfloat16)
+        idx = torch.empty((cap,), dtype=torch.int32, device=dev)
+        n_out = torch.empty((1,), dtype=torch.int32, device=dev)
+        Xo = torch.empty((Mq, cap), dtype=torch.bfloat16, device=dev)
+        split = lambda i: W.int8_outlier_split(Xl, case.threshold, cap, Xq=Xq, S_x=S, idx=idx, n_out=n_out, Xo=Xo,
+                                               workspace=wsb)
+        split_us = graph_time_us(split, 4)
+        n = int(n_out.item())
+        cuda_us = graph_time_us(lambda i: W.int8_mixed_decomp_gemm(Xq, S, Xo, idx, n_out, cap, Wq, s_w, Wd, out=out),
+                                4, reps=3 if n > 64 else 10)
+        tc_us = graph_time_us(lambda i: W.int8_mixed_decomp_gemm_tc(Xq, S, Xo, idx, n_out, cap, Wq, s_w, Wd, out=out), 4)
+        split_bytes = 2.0 * Mq * Kq + Mq * Kq + 4.0 * Mq + 2.0 * Mq * n
+        res["rows"].append({"outlier_columns": n, "cap": cap,
+                            "split_us": split_us, "split_GB/s": split_bytes / (split_us * 1e-6) / 1e9,
+                            "split_frac_hbm": split_bytes / (split_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                            "mixed_cuda_core_side_us": cuda_us,
+                            "mixed_cuda_core_side_frac_int8": ops / (cuda_us * 1e-6) / 1e12 / int8_peak,
+                            "mixed_tensor_core_side_us": tc_us,
+                            "mixed_tensor_core_side_frac_int8": ops / (tc_us * 1e-6) / 1e12 / int8_peak})
+        if label == "workload":
+            res.update({"outlier_columns": n, "split_us": split_us,
+                        "split_frac_hbm": res["rows"][0]["split_frac_hbm"], "split_algorithmic_bytes": split_bytes})
+        del Xl
+    # the plain pair GEMM of the same shape (no side product), for the overhead of the side path
+    plain_us = graph_time_us(lambda i: W.w8a8_gemm_dequant(Xq, S, Wq, s_w, out=out), 4)
+    res["plain_gemm_us"] = plain_us
+    res["plain_gemm_frac_int8"] = ops / (plain_us * 1e-6) / 1e12 / int8_peak
+    for r in res["rows"]:
+        r["tensor_core_side_over_plain"] = r["mixed_tensor_core_side_us"] / plain_us
+        r["cuda_core_side_over_plain"] = r["mixed_cuda_core_side_us"] / plain_us
     assert W.w8a8_check_device_error() == 0
-    return {"workload": f"LLM.int8() X [{Mq} x {Kq}] ({int(n_out.item())} outlier columns), W bf16 [{Kq} x {Nq}], threshold 6.0",
-            "split_us": split_us, "split_GB/s": split_bytes / (split_us * 1e-6) / 1e9,
-            "split_frac_hbm": split_bytes / (split_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
-            "split_algorithmic_bytes": split_bytes,
-            "mixed_gemm_us": gemm_us, "mixed_gemm_TOPS": ops / (gemm_us * 1e-6) / 1e12,
-            "mixed_gemm_frac_int8": ops / (gemm_us * 1e-6) / 1e12 / int8_peak}
+    return res
 
 
 def bench_block(args, dev, rank, peaks, int8_peak):
@@ -656,6 +790,8 @@ def main(argv=None):
     ap.add_argument("--no-block", action="store_true")
     ap.add_argument("--no-quant-stream", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sustained", action="store_true")
+    ap.add_argument("--no-c1", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=16)
     args = ap.parse_args(argv)
