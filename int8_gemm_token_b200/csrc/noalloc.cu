@@ -2,10 +2,9 @@
 // caller-provided workspace.
 //
 // Some callers cannot allocate device memory at the point where they run a
-// Decode step: a serving loop whose CUDA graph is being captured (cudaMalloc
-// is not a stream operation and breaks the capture), a plug-in running inside
-// another runtime that owns all device memory, or a latency-critical step
-// where an allocation's implicit device synchronization is not acceptable.
+// Decode step: a plug-in running inside another runtime that owns all device
+// memory and hands none out, or a latency-critical step where the
+// device-wide synchronization an allocation may cause is not acceptable.
 // This entry point needs no memory from them: its scratch (the statically
 // quantized activation handed from the quantization kernel to the GEMM)
 // lives in one file-scope device array of fixed size, which every GPU that
