@@ -375,14 +375,24 @@ w8a8_status int8_mixed_decomp_gemm(const int8_t *Xq, const float *S_x, const voi
  * the mixed-precision decomposition formula Y. Reading: the pages' FP16 side
  * GEMM is taken as bf16 inputs with fp32 accumulation, as in
  * int8_mixed_decomp_gemm.
+ *   workspace  device, >= int8_mixed_decomp_gemm_tc_workspace_size(M, N, cap)
+ *              bytes, 16-byte aligned: the side operands, zero-padded to
+ *              whole blocks of 64 outlier columns, written by the call (no
+ *              initial contents needed; calls that overlap on the GPU must
+ *              not share it).
  * Any M; Xo and W 16-byte aligned; the columns of Xo at or past n_used are
- * not read.
+ * not read. Errors as int8_mixed_decomp_gemm, plus W8A8_ERR_WORKSPACE.
  */
 w8a8_status int8_mixed_decomp_gemm_tc(const int8_t *Xq, const float *S_x, const void *Xo,
                                       const int32_t *outlier_idx, const int32_t *n_out, int32_t cap,
                                       const int8_t *Wq, const float *s_w, const void *W, int64_t ldw,
                                       const float *bias, int64_t M, int64_t N, int64_t K, void *out,
-                                      w8a8_dtype out_dtype, void *stream);
+                                      w8a8_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                                      void *stream);
+
+/* Bytes of device workspace int8_mixed_decomp_gemm_tc needs: (M + N) rows of
+ * cap rounded up to a multiple of 64 bf16 values (0 for a bad shape). */
+size_t int8_mixed_decomp_gemm_tc_workspace_size(int64_t M, int64_t N, int32_t cap);
 
 /*
  * Device status word. Kernels record device-side failures (a bounded wait

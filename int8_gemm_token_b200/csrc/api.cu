@@ -113,7 +113,10 @@ bool encode_tmap_2d(void *map, const void *base, TmapType type, uint64_t inner, 
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(static_cast<CUtensorMap *>(map),
-                        type == TmapType::kU8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        type == TmapType::kU8    ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                        : type == TmapType::kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        2,
                         const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -433,20 +436,29 @@ static w8a8_status check_mixed(const int8_t *Xq, const float *S_x, const void *X
   return W8A8_OK;
 }
 
+size_t int8_mixed_decomp_gemm_tc_workspace_size(int64_t M, int64_t N, int32_t cap) {
+  if (M <= 0 || N <= 0 || cap < 0 || cap > 4096) return 0;
+  return align256(static_cast<int64_t>(side_workspace_bytes(M, N, cap)));
+}
+
 w8a8_status int8_mixed_decomp_gemm_tc(const int8_t *Xq, const float *S_x, const void *Xo,
                                       const int32_t *outlier_idx, const int32_t *n_out, int32_t cap,
                                       const int8_t *Wq, const float *s_w, const void *W, int64_t ldw,
                                       const float *bias, int64_t M, int64_t N, int64_t K, void *out,
-                                      w8a8_dtype out_dtype, void *stream) {
+                                      w8a8_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                                      void *stream) {
   EpilogueArgs ep;
   if (w8a8_status s = check_mixed(Xq, S_x, Xo, outlier_idx, n_out, cap, Wq, s_w, W, ldw, bias, M, N, K, out,
                                   out_dtype, &ep))
     return s;
   if (M == 0 || N == 0) return W8A8_OK;
+  if (!workspace || workspace_bytes < int8_mixed_decomp_gemm_tc_workspace_size(M, N, cap))
+    return W8A8_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return W8A8_ERR_MISALIGNED;
   DeviceInfo *d;
   if (w8a8_status s = device_info(&d)) return s;
   if (d->sm_count < 2) return W8A8_ERR_NO_DEVICE;
-  return from_cuda(launch_gemm_side_tc(Xq, Wq, M, N, K, ep, d->sm_count, d->status,
+  return from_cuda(launch_gemm_side_tc(Xq, Wq, M, N, K, ep, workspace, d->sm_count, d->status,
                                        static_cast<cudaStream_t>(stream)));
 }
 

@@ -17,6 +17,40 @@ struct PairExitWords {
   volatile int *peer_abort;  // leader: rank 1's producer gave up
 };
 
+// Exit of a pair producer (one thread per CTA) whose copies all complete on
+// the leader's `full_bar` ring of STAGES stages, `half_bytes` per CTA per
+// fill; `fills` counts the fills this CTA issued. Rank 1 reports its count
+// and whether it gave up; after a failure in either CTA the leader
+// reconciles each stage's last fill -- completing the half of a fill that
+// rank 1 never issued, or arming the half that only rank 1 issued -- and
+// waits (bounded) for it, so that no CTA leaves while a copy into its shared
+// memory may still be in flight.
+template <int STAGES>
+__device__ __forceinline__ void pair_producer_exit(uint32_t rank, int fills, bool ok, uint64_t *full_bar,
+                                                   const PairExitWords &xw, volatile int *abort_flag,
+                                                   uint32_t half_bytes, int32_t *status, uint64_t limit_ns) {
+  if (rank != 0) {
+    st_shared_cluster(map_to_rank(const_cast<int *>(xw.peer_fills), 0), static_cast<uint32_t>(fills));
+    st_shared_cluster(map_to_rank(const_cast<int *>(xw.peer_abort), 0), ok ? 0u : 1u);
+    mbar_arrive_remote(map_to_rank(xw.exit_bar, 0));
+    return;
+  }
+  const bool heard = mbar_wait_bounded_cluster(xw.exit_bar, 0, nullptr, limit_ns);
+  if (heard && !*xw.peer_abort && !*abort_flag) return;
+  if (!heard) record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
+  const int fr = heard ? *xw.peer_fills : fills;  // unheard: assume rank 1 matched the leader
+  for (int s = 0; s < STAGES; ++s) {
+    // last fill of stage s by each CTA (-1: none); they differ by at most one ring turn
+    const int fl = fills > s ? s + ((fills - 1 - s) / STAGES) * STAGES : -1;
+    const int fp = fr > s ? s + ((fr - 1 - s) / STAGES) * STAGES : -1;
+    const int f = fl > fp ? fl : fp;
+    if (f < 0) continue;
+    if (fl > fp) mbar_complete_tx(&full_bar[s], half_bytes);      // rank 1's half never comes
+    if (fp > fl) mbar_arrive_expect_tx(&full_bar[s], half_bytes);  // only rank 1's half comes
+    mbar_wait_bounded(&full_bar[s], static_cast<uint32_t>(f / STAGES) & 1u, nullptr, limit_ns / 16 + 1);
+  }
+}
+
 // Run by one thread (lane 0 of the producer warp) of each CTA of the pair.
 // Tile t covers rows (t % num_m) * 256 + [0, 256) of Xq and rows
 // (t / num_m) * 256 + [0, 256) of Wq; CTA `rank` loads the 128 rows
@@ -82,27 +116,7 @@ __device__ __forceinline__ void pair_tma_producer(const CUtensorMap *tmA, const 
     record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
     *abort_flag = 1;
   }
-  if (!leader) {
-    st_shared_cluster(map_to_rank(const_cast<int *>(xw.peer_fills), 0), static_cast<uint32_t>(fills));
-    st_shared_cluster(map_to_rank(const_cast<int *>(xw.peer_abort), 0), ok ? 0u : 1u);
-    mbar_arrive_remote(map_to_rank(xw.exit_bar, 0));
-    return;
-  }
-  const bool heard = mbar_wait_bounded(xw.exit_bar, 0, nullptr, limit_ns);
-  fence_acq_rel_cluster();
-  if (heard && !*xw.peer_abort && !*abort_flag) return;
-  if (!heard) record_error(status, W8A8_ERR_DEVICE_TIMEOUT);
-  const int fr = heard ? *xw.peer_fills : fills;  // unheard: assume rank 1 matched the leader
-  for (int s = 0; s < STAGES; ++s) {
-    // last fill of stage s by each CTA (-1: none); they differ by at most one ring turn
-    const int fl = fills > s ? s + ((fills - 1 - s) / STAGES) * STAGES : -1;
-    const int fp = fr > s ? s + ((fr - 1 - s) / STAGES) * STAGES : -1;
-    const int f = fl > fp ? fl : fp;
-    if (f < 0) continue;
-    if (fl > fp) mbar_complete_tx(&full_bar[s], kStageA2 + kStageB2);      // rank 1's half never comes
-    if (fp > fl) mbar_arrive_expect_tx(&full_bar[s], kStageA2 + kStageB2);  // only rank 1's half comes
-    mbar_wait_bounded(&full_bar[s], static_cast<uint32_t>(f / STAGES) & 1u, nullptr, limit_ns / 16 + 1);
-  }
+  pair_producer_exit<STAGES>(rank, fills, ok, full_bar, xw, abort_flag, kStageA2 + kStageB2, status, limit_ns);
 }
 
 }  // namespace w8a8

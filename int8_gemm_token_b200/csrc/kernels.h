@@ -82,9 +82,13 @@ cudaError_t launch_gemm_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_
                            cudaStream_t s);
 
 // LLM.int8() mixed GEMM with the 16-bit side product on the tensor cores
-// (CTA pairs, one int32 and one fp32 TMEM accumulator per tile; any M).
+// (CTA pairs, one int32 and one fp32 TMEM accumulator per tile; any M). A
+// gather kernel first writes the side operands, zero-padded to whole 64-column
+// k-blocks, into `workspace` (side_workspace_bytes(M, N, cap) bytes).
 cudaError_t launch_gemm_side_tc(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
-                                const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s);
+                                const EpilogueArgs &ep, void *workspace, int num_sms, int32_t *status,
+                                cudaStream_t s);
+size_t side_workspace_bytes(int64_t M, int64_t N, int32_t cap);
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *status, cudaStream_t s);
 
@@ -121,7 +125,7 @@ w8a8_status current_device_info(int *sm_count, int32_t **status_word);
 // 2-D tensor map (driver entry point resolved once per process): inner and
 // outer extents in elements, row stride in bytes, box in elements; swizzle128
 // selects the 128-byte swizzle (box inner extent must then be 128 bytes).
-enum class TmapType { kU8, kBF16 };
+enum class TmapType { kU8, kBF16, kF32 };
 bool encode_tmap_2d(void *map, const void *base, TmapType type, uint64_t inner, uint64_t outer,
                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
 

@@ -54,7 +54,8 @@ _SIGNATURES = {
     "int8_outlier_split_workspace_size": (_SZ, [_I64]),
     "int8_mixed_decomp_gemm": (_I32, [_P, _P, _P, _P, _P, _I32, _P, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _I32, _P]),
     "int8_mixed_decomp_gemm_tc": (_I32, [_P, _P, _P, _P, _P, _I32, _P, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _I32,
-                                         _P]),
+                                         _P, _SZ, _P]),
+    "int8_mixed_decomp_gemm_tc_workspace_size": (_SZ, [_I64, _I64, _I32]),
     "w8a8_check_device_error": (_I32, [_P, _P]),
     "w8a8_debug_wait_timeout_selftest": (_I32, [ctypes.c_uint64, _P]),
 }
@@ -429,7 +430,7 @@ def int8_outlier_split(X, threshold: float = 6.0, cap: int = 64, Xq=None, S_x=No
     return Xq, S_x, idx, n_out, Xo
 
 
-def _mixed(fn, Xq, S_x, Xo, idx, n_out, cap, Wq, s_w, W, bias, out, out_dtype, stream):
+def _mixed(fn, Xq, S_x, Xo, idx, n_out, cap, Wq, s_w, W, bias, out, out_dtype, stream, workspace=None):
     if Xq.dtype != torch.int8 or Xq.dim() != 2:
         raise ValueError(f"Xq: expected a 2-D int8 tensor, got {Xq.dtype} {tuple(Xq.shape)}")
     M, K = Xq.shape
@@ -443,10 +444,14 @@ def _mixed(fn, Xq, S_x, Xo, idx, n_out, cap, Wq, s_w, W, bias, out, out_dtype, s
     _vec(n_out, torch.int32, 1, "n_out")
     ldw = _rows(W, torch.bfloat16, "W", shape=(K, N))
     out = _out(out, out_dtype, (M, N), Xq.device, (torch.bfloat16, torch.float32))
-    _on_one_gpu(Xq, S_x, Xo, idx, n_out, Wq, s_w, W, bias, out)
-    _check(fn, getattr(lib(), fn)(
-        _ptr(Xq), _ptr(S_x), _ptr(Xo), _ptr(idx), _ptr(n_out), cap, _ptr(Wq), _ptr(s_w), _ptr(W),
-        ldw, _ptr(bias), M, N, K, _ptr(out), _dt(out.dtype), _stream(stream)))
+    args = [_ptr(Xq), _ptr(S_x), _ptr(Xo), _ptr(idx), _ptr(n_out), cap, _ptr(Wq), _ptr(s_w), _ptr(W),
+            ldw, _ptr(bias), M, N, K, _ptr(out), _dt(out.dtype)]
+    ws = None
+    if fn == "int8_mixed_decomp_gemm_tc":
+        ws, nbytes = _workspace(int(lib().int8_mixed_decomp_gemm_tc_workspace_size(M, N, cap)), Xq.device, workspace)
+        args += [_ptr(ws), nbytes]
+    _on_one_gpu(Xq, S_x, Xo, idx, n_out, Wq, s_w, W, bias, out, ws)
+    _check(fn, getattr(lib(), fn)(*args, _stream(stream)))
     return out
 
 
@@ -458,11 +463,12 @@ def int8_mixed_decomp_gemm(Xq, S_x, Xo, idx, n_out, cap: int, Wq, s_w, W, bias=N
 
 
 def int8_mixed_decomp_gemm_tc(Xq, S_x, Xo, idx, n_out, cap: int, Wq, s_w, W, bias=None, out=None,
-                              out_dtype=torch.bfloat16, stream=None):
+                              out_dtype=torch.bfloat16, workspace=None, stream=None):
     """The same decomposition with the bf16 side product on the tensor cores
-    (kind::f16 MMAs into a second TMEM accumulator)."""
+    (kind::f16 MMAs into a second TMEM accumulator); `workspace` (allocated
+    when None) holds the padded side operands."""
     return _mixed("int8_mixed_decomp_gemm_tc", Xq, S_x, Xo, idx, n_out, cap, Wq, s_w, W, bias, out, out_dtype,
-                  stream)
+                  stream, workspace)
 
 
 def w8a8_check_device_error(stream=None) -> int:
