@@ -29,11 +29,16 @@
 //                 accumulator;
 //     warp 2      TMA producer of the side k-blocks (XoP and WoT boxes of
 //                 64 columns x 128 rows, a two-stage ring);
-//     warps 4..7  epilogue: tcgen05.ld of both accumulators (the next 32
-//                 columns in flight), the fixed-order fp32 epilogue, and the
-//                 results staged per warp in 128B-swizzled shared memory and
-//                 written by TMA tensor stores; the accumulators go back to
-//                 the MMAs as soon as they are read.
+//     warps 4..11 epilogue, two warps per TMEM lane quarter (warp w reads
+//                 lanes 32 (w % 4) ..), each with 128 of the tile's 256
+//                 columns: tcgen05.ld of both accumulators, the fixed-order
+//                 fp32 epilogue, and the results staged per warp in
+//                 128B-swizzled shared memory and written by TMA tensor
+//                 stores; the accumulators go back to the MMAs as soon as
+//                 every warp has read its part. With the accumulators single
+//                 buffered, this phase is not overlapped with the next tile's
+//                 MMAs; two warps per SM sub-partition hide each other's
+//                 load latencies.
 // Every wait is bounded; on a timeout the CTA records
 // W8A8_ERR_DEVICE_TIMEOUT, stops, lets its copies and MMAs in flight finish,
 // frees its TMEM and returns.
@@ -45,8 +50,9 @@ namespace w8a8 {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each with half of the tile's columns
 constexpr int kBK = 128;             // bytes of K per INT8 k-block
 constexpr int kHalf = 128;           // rows of A and of B per CTA
 constexpr int kStage2 = kHalf * kBK; // 16 KiB per operand per stage
@@ -62,7 +68,7 @@ constexpr int kStages = 4;                   // INT8 ring depth
 struct SideSmem {
   static constexpr size_t kRing = static_cast<size_t>(kStages) * 2 * kStage2;
   static constexpr size_t kSide = static_cast<size_t>(kSideStages) * kSideStage;
-  static constexpr size_t kStage = 4 * kStaging;
+  static constexpr size_t kStage = kEpiWarps * kStaging;
   static constexpr size_t kBytes = kRing + kSide + kStage + 1024 /*alignment slack*/ + 256 /*barriers, flags*/;
   static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
   static_assert((2 * kStages + 2 * kSideStages + 5) * 8 + 7 * 4 <= 256, "barriers and flags fit their reserve");
@@ -268,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *sfull_bar = empty_bar + kStages;       // leader: both CTAs' side boxes landed
   uint64_t *sempty_bar = sfull_bar + kSideStages;  // the side MMAs reading the stage completed
   uint64_t *tfull_bar = sempty_bar + kSideStages;  // both accumulators of the tile are final
-  uint64_t *tempty_bar = tfull_bar + 1;            // leader: both CTAs' epilogues have read them (8 arrivals)
+  uint64_t *tempty_bar = tfull_bar + 1;            // leader: both CTAs' epilogues have read them (16 arrivals)
   uint64_t *drain_bar = tempty_bar + 1;
   uint64_t *exit_bar = drain_bar + 1;              // leader: INT8 producer handshake
   uint64_t *sexit_bar = exit_bar + 1;              // leader: side producer handshake
@@ -296,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sempty_bar[s], 1);
     }
     mbar_init(tfull_bar, 1);
-    mbar_init(tempty_bar, 8);
+    mbar_init(tempty_bar, 2 * kEpiWarps);  // every epilogue warp of both CTAs
     mbar_init(drain_bar, 1);
     mbar_init(exit_bar, 1);
     mbar_init(sexit_bar, 1);
@@ -436,11 +442,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kEpiWarp0) {
     // -------------------------------------------------- epilogue (both CTAs)
     pdl_wait_prerequisite();  // S_x, s_w, bias, n_out and `out` belong to the previous kernels until then
-    const int q = warp - kEpiWarp0;
+    const int e = warp - kEpiWarp0;   // 0..7
+    const int q = warp & 3;           // TMEM lane quarter this warp may read
+    const int h = e >> 2;             // column half: [128 h, 128 h + 128)
     const int nuse = min(__ldg(ep.n_out), ep.cap);
     const bool has_side = nuse > 0;
     const bool bf16 = ep.out_dtype == W8A8_BF16;
-    uint8_t *stage = sStage + q * kStaging;
+    uint8_t *stage = sStage + e * kStaging;
     uint32_t tphase = 0;
     for (int64_t tile = cluster_id; tile < num_tiles; tile += num_clusters) {
       if (*abort_flag) break;
@@ -455,32 +463,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int64_t mrow0 = (tile % num_m) * kTileM + rank * kHalf + q * 32;  // this warp's first row
       const int64_t m = mrow0 + lane;
-      const int64_t ntile = (tile / num_m) * kTileN;
+      const int64_t ncol0 = (tile / num_m) * kTileN + 128 * h;                 // this warp's first column
       const float sx = m < M ? __ldg(ep.S_x + m) : 0.0f;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      uint32_t ra[32], rs[32], rb[32], rt[32];
-      tmem_ld_32x32b_x32(taddr, ra);
-      if (has_side) tmem_ld_32x32b_x32(taddr + kSideCol, rs);
-#pragma unroll
-      for (int c = 0; c < kTileN / 32; c += 2) {
-        float y[32];
-        tmem_ld_wait();  // chunk c in ra / rs; request chunk c + 1 before converting chunk c
-        tmem_ld_32x32b_x32(taddr + (c + 1) * 32, rb);
-        if (has_side) tmem_ld_32x32b_x32(taddr + kSideCol + (c + 1) * 32, rt);
-        side_epilogue_values(ra, rs, has_side, ntile + c * 32, N, sx, ep, y);
-        if (tma_store) {
-          stage_free(lane);
-          stage_row32(y, stage, lane, 0, bf16);
-          if (!bf16) flush_stage(&tmOut, stage, lane, ntile + c * 32, mrow0);  // fp32: 32 columns fill the rows
-        } else {
-          store_row32(y, m, ntile + c * 32, M, N, ep);
-        }
-        tmem_ld_wait();  // chunk c + 1 in rb / rt
-        if (c + 2 < kTileN / 32) {
-          tmem_ld_32x32b_x32(taddr + (c + 2) * 32, ra);
-          if (has_side) tmem_ld_32x32b_x32(taddr + kSideCol + (c + 2) * 32, rs);
-        } else {
-          // every accumulator column of the tile is in registers: hand TMEM back to the MMAs
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(128 * h);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ra[32], rs[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, ra);
+        if (has_side) tmem_ld_32x32b_x32(taddr + kSideCol + c * 32, rs);
+        tmem_ld_wait();
+        if (c == 3) {  // every accumulator column of this warp is in registers: hand TMEM back
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
@@ -490,18 +482,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_remote(map_to_rank(tempty_bar, 0));
           }
         }
-        side_epilogue_values(rb, rt, has_side, ntile + (c + 1) * 32, N, sx, ep, y);
-        if (tma_store) {
-          if (bf16) {  // the second half of the 64 staged bf16 columns, then one store of both chunks
-            stage_row32(y, stage, lane, 1, true);
-            flush_stage(&tmOut, stage, lane, ntile + c * 32, mrow0);
-          } else {
-            stage_free(lane);
-            stage_row32(y, stage, lane, 0, false);
-            flush_stage(&tmOut, stage, lane, ntile + (c + 1) * 32, mrow0);
-          }
-        } else {
-          store_row32(y, m, ntile + (c + 1) * 32, M, N, ep);
+        float y[32];
+        side_epilogue_values(ra, rs, has_side, ncol0 + c * 32, N, sx, ep, y);
+        if (!tma_store) {
+          store_row32(y, m, ncol0 + c * 32, M, N, ep);
+        } else if (bf16) {  // two chunks (64 bf16 columns) per staged box
+          if ((c & 1) == 0) stage_free(lane);
+          stage_row32(y, stage, lane, c & 1, true);
+          if (c & 1) flush_stage(&tmOut, stage, lane, ncol0 + (c - 1) * 32, mrow0);
+        } else {  // fp32: one chunk (32 columns) per staged box
+          stage_free(lane);
+          stage_row32(y, stage, lane, 0, false);
+          flush_stage(&tmOut, stage, lane, ncol0 + c * 32, mrow0);
         }
       }
       tphase ^= 1u;
