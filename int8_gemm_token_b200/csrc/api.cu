@@ -177,6 +177,10 @@ w8a8_status w8a8_calibrate_static(const void *Xcal, w8a8_dtype x_dtype, int64_t 
                                     static_cast<cudaStream_t>(stream)));
 }
 
+// Dense tensors of at least this many elements take the streaming kernels
+// (stream.cu); below it a single grid-stride launch finishes sooner.
+constexpr int64_t kStreamMinElems = int64_t(1) << 22;
+
 w8a8_status w8a8_quant_per_token(const void *X, int64_t M, int64_t K, int64_t ldx, int8_t *Xq,
                                  float *S_x, void *stream) {
   if (w8a8_status s = check_bf16_rows(X, M, K, ldx)) return s;
@@ -197,6 +201,9 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
   if ((reinterpret_cast<uintptr_t>(Xq) & 15u) != 0) return W8A8_ERR_MISALIGNED;
   DeviceInfo *d;
   if (w8a8_status s = device_info(&d)) return s;
+  if (ldx == K && M * K >= kStreamMinElems)  // a large dense tensor: streamed through shared memory
+    return from_cuda(launch_quant_per_tensor_stream(static_cast<const uint16_t *>(X), M * K, r, Z, Xq, d->sm_count,
+                                                    d->status, static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_quant_per_tensor(static_cast<const uint16_t *>(X), M, K, ldx, r, Z, Xq,
                                            d->sm_count, static_cast<cudaStream_t>(stream), /*pdl=*/true));
 }
@@ -212,6 +219,9 @@ w8a8_status w8a8_dequant_per_tensor(const int8_t *Xq, int64_t M, int64_t K, int6
   if (!aligned16(Xq) || (ldq % 16) != 0 || !aligned16(out)) return W8A8_ERR_MISALIGNED;
   DeviceInfo *d;
   if (w8a8_status s = device_info(&d)) return s;
+  if (ldq == K && M * K >= kStreamMinElems)
+    return from_cuda(launch_dequant_per_tensor_stream(Xq, M * K, S, Z, out, out_dtype == W8A8_BF16, d->sm_count,
+                                                      d->status, static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_dequant_per_tensor(Xq, M, K, ldq, S, Z, out, out_dtype == W8A8_BF16, d->sm_count,
                                              static_cast<cudaStream_t>(stream)));
 }

@@ -70,6 +70,13 @@ cudaError_t launch_quant_per_tensor(const uint16_t *X, int64_t M, int64_t K, int
 // out [M, K] dense = S * (Xq - Z) as bf16 (bf16_out) or fp32; K a multiple of 16.
 cudaError_t launch_dequant_per_tensor(const int8_t *Xq, int64_t M, int64_t K, int64_t ldq, const float *S,
                                       const int32_t *Z, void *out, bool bf16_out, int num_sms, cudaStream_t s);
+// The same two conversions for large dense tensors (rows of exactly K
+// elements), streamed through shared memory with bulk copies (stream.cu).
+cudaError_t launch_quant_per_tensor_stream(const uint16_t *X, int64_t elems, const float *r, const int32_t *Z,
+                                           int8_t *Xq, int num_sms, int32_t *status, cudaStream_t s);
+cudaError_t launch_dequant_per_tensor_stream(const int8_t *Xq, int64_t elems, const float *S, const int32_t *Z,
+                                             void *out, bool bf16_out, int num_sms, int32_t *status,
+                                             cudaStream_t s);
 cudaError_t launch_calibrate(const void *X, w8a8_dtype dt, int64_t T, int64_t K, int64_t ldx,
                              float *S, float *r, int32_t *Z, int num_sms, cudaStream_t s);
 cudaError_t launch_quant_weight(const void *W, w8a8_dtype dt, int64_t K, int64_t N, int64_t ldw,

@@ -549,3 +549,23 @@ def test_kv_cache_round_trip(M, K):
     rq = oracle.quant_per_tensor(X, rr, rZ)
     assert_same(host(q), rq, "codes")
     assert_same(host_bf16(back), oracle.dequant_per_tensor(rq, rS, rZ), "values")
+
+
+@pytest.mark.parametrize("M,K", [(4099, 1040), (2048, 2048)])
+def test_static_quant_and_dequant_stream_path_bit_exact(M, K):
+    """Dense tensors of 4M elements or more take the kernels that stream
+    16 KiB tiles through shared memory with bulk copies: codes and values
+    equal the oracle's, with every finite bf16 value in the input and a
+    total size (4099 x 1040) that is not a whole number of tiles."""
+    finite = _all_finite_bf16(1).reshape(-1)
+    reps = -(-(M * K) // finite.size)
+    X = np.tile(finite, reps)[:M * K].reshape(M, K)
+    case = synth.decode_static(M=1, N=16, K=K, seed=M)
+    S, r, Z = W.w8a8_calibrate_static(dev_bf16(case.Xcal))
+    rS, rr, rZ = oracle.calibrate_static(case.Xcal)
+    q = W.w8a8_quant_per_tensor(dev_bf16(X), r, Z)
+    rq = oracle.quant_per_tensor(X, rr, rZ)
+    assert_same(host(q), rq, "codes")
+    assert_same(host_bf16(W.w8a8_dequant_per_tensor(q, S, Z)), oracle.dequant_per_tensor(rq, rS, rZ), "bf16 values")
+    assert_same(host(W.w8a8_dequant_per_tensor(q, S, Z, out_dtype=torch.float32)),
+                oracle.dequant_per_tensor(rq, rS, rZ, oracle.DT_FP32), "fp32 values")
