@@ -453,11 +453,11 @@ __device__ __forceinline__ uint2 quant8_sym_sat(const uint4 &v, float r) {
   return make_uint2(pack_sat_s8x4(q[0], q[1], q[2], q[3]), pack_sat_s8x4(q[4], q[5], q[6], q[7]));
 }
 
-// Low bytes of four int32, a in the lowest byte.
-__device__ __forceinline__ uint32_t pack_i8x4(int a, int b, int c, int d) {
-  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+// The low bytes of four words, a in the lowest byte (two byte permutes).
+__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
+
 
 // rne(y) held to [-1024, 1024] on the full-rate FP32 and integer pipes: adding
 // 1.5 * 2^23 to a value of magnitude <= 2^22 leaves it rounded to the nearest
@@ -477,9 +477,9 @@ __device__ __forceinline__ uint2 quant8_asym_sat(const uint4 &v, float r, int z)
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     q[2 * i] = min(max(rne_held(__fmul_rn(bf16_lo(w[i]), r)) + z, -128), 127);
-    q[2 * i + 1] = min(max(rne_held(__fmul_rn(bf16_hi(w[i]), r)) + z, -128), 127);
+    q[2 * i + 1] = min(max(rne_held(__fmul_rn(bf16_hi(w[i]), r)) + z, -128), 127);  // low bytes: the codes
   }
-  return make_uint2(pack_i8x4(q[0], q[1], q[2], q[3]), pack_i8x4(q[4], q[5], q[6], q[7]));
+  return make_uint2(low_bytes4(q[0], q[1], q[2], q[3]), low_bytes4(q[4], q[5], q[6], q[7]));
 }
 
 // Running per-halfword maximum of bf16 magnitudes (two values per word).

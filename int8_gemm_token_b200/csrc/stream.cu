@@ -14,7 +14,8 @@
 // grid of one CTA per SM; in each, one thread (the producer) copies 16 KiB
 // tiles of the input with 1-D bulk copies (cp.async.bulk, completion on an
 // mbarrier) into an 8-stage shared-memory ring -- 128 KiB in flight per SM
-// -- and four consumer warps convert each tile from shared memory and store
+// -- and consumer warps (eight for the quantization, four for the
+// dequantization) convert each tile from shared memory and store
 // the results to global memory (coalesced 8- to 64-byte stores per thread),
 // then release the stage. Tiles are dealt to the CTAs round robin.
 // Programmatic dependent launch: the kernel lets its dependents launch at
@@ -30,8 +31,10 @@ namespace {
 
 constexpr int kTile = 16384;  // input bytes per stage
 constexpr int kStages = 8;
-constexpr int kConsumers = 4;  // warps
-constexpr int kThreads = 32 * (1 + kConsumers);
+// Consumer warps per CTA: the quantization's per-byte arithmetic needs two
+// per SM sub-partition to hide its latency; the dequantization, one.
+template <int Cw>
+constexpr int threads_for() { return 32 * (1 + Cw); }
 constexpr size_t kSmem = static_cast<size_t>(kStages) * kTile + 2 * kStages * 8 + 16 + 128;
 
 enum class Conv { kQuant, kDequantBf16, kDequantF32 };
@@ -67,11 +70,15 @@ __device__ __forceinline__ void convert_piece(const uint4 &v, int64_t e, void *o
 // element count. a, z: r and Z (quantization) or S and Z (dequantization),
 // device scalars.
 template <Conv C>
-__global__ void __launch_bounds__(kThreads, 1)
+constexpr int consumers_for() { return C == Conv::kQuant ? 8 : 4; }
+
+template <Conv C>
+__global__ void __launch_bounds__(threads_for<consumers_for<C>()>(), 1)
     stream_convert_kernel(const uint8_t *__restrict__ in, int64_t in_bytes, void *__restrict__ out,
                           const float *__restrict__ a_ptr, const int32_t *__restrict__ z_ptr, int32_t *status,
                           uint64_t limit_ns) {
   constexpr int kElem = C == Conv::kQuant ? 2 : 1;  // input bytes per element
+  constexpr int kConsumers = consumers_for<C>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *ring = smem_raw;
   uint64_t *full_bar = reinterpret_cast<uint64_t *>(ring + static_cast<size_t>(kStages) * kTile);
@@ -130,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait_prerequisite();  // the scalars (and `out`) belong to the previous kernel until then
   const float a = __ldg(a_ptr);
   const int z = __ldg(z_ptr);
-  const int ct = threadIdx.x - 32;  // 0 .. 127
+  const int ct = threadIdx.x - 32;  // 0 .. 32 * kConsumers - 1
   int i = 0;
   for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
     const int s = i % kStages;
@@ -162,7 +169,7 @@ cudaError_t launch_stream_t(const void *in, int64_t in_bytes, void *out, const f
   const int64_t n_tiles = (in_bytes + kTile - 1) / kTile;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(n_tiles < num_sms ? n_tiles : num_sms));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(threads_for<consumers_for<C>()>());
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
