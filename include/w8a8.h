@@ -123,7 +123,10 @@ w8a8_status w8a8_quant_per_token(const void *X, int64_t M, int64_t K, int64_t ld
  * Source: PDMIX glossary §2.3 eq. Q_decode; the saturation it implies for
  * out-of-range tokens is the risk named in §2.4.
  * Xq[m, k] = clamp(rne(X[m, k] * r) + Z, -128, 127), r and Z from
- * w8a8_calibrate_static (device scalars, read by the kernel).
+ * w8a8_calibrate_static (device scalars, read by the kernel). Z is an int8
+ * zero point, in [-128, 127] as w8a8_calibrate_static writes it; the result
+ * for a Z outside that range is unspecified (the kernel cannot check a
+ * device scalar without a synchronisation).
  *   X   device bf16 [M, K], row stride ldx;  Xq device int8 [M, K] dense, written
  */
 w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t ldx, const float *r,
@@ -143,6 +146,7 @@ w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t l
  * Decode scheme is taken.
  *   Xq   device int8 [M, K], row stride ldq bytes (a multiple of 16)
  *   S, Z device scalars (fp32, int32), as from w8a8_calibrate_static
+ *        (Z in [-128, 127]; outside it the result is unspecified)
  *   out  device [M, K] dense, 16-byte aligned, written
  */
 w8a8_status w8a8_dequant_per_tensor(const int8_t *Xq, int64_t M, int64_t K, int64_t ldq, const float *S,

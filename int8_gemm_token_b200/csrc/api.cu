@@ -189,7 +189,7 @@ w8a8_status w8a8_quant_per_token(const void *X, int64_t M, int64_t K, int64_t ld
   if ((reinterpret_cast<uintptr_t>(Xq) & 15u) != 0) return W8A8_ERR_MISALIGNED;
   DeviceInfo *d;
   if (w8a8_status s = device_info(&d)) return s;
-  return from_cuda(launch_quant_per_token(static_cast<const uint16_t *>(X), M, K, ldx, Xq, S_x,
+  return from_cuda(launch_quant_per_token(static_cast<const uint16_t *>(X), M, K, ldx, Xq, S_x, d->sm_count,
                                           static_cast<cudaStream_t>(stream)));
 }
 

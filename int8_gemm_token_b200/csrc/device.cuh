@@ -459,27 +459,52 @@ __device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t 
 }
 
 
-// rne(y) held to [-1024, 1024] on the full-rate FP32 and integer pipes: adding
-// 1.5 * 2^23 to a value of magnitude <= 2^22 leaves it rounded to the nearest
-// integer, ties to even, in the low mantissa bits.
-__device__ __forceinline__ int rne_held(float y) {
-  y = fminf(fmaxf(y, -1024.0f), 1024.0f);
-  return __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
-}
-
 // Static asymmetric codes of the 8 bf16 values in one uint4:
-// clamp(rne(x * r) + Z, -128, 127). Holding the rounded value to
-// [-1024, 1024] first is invisible after the final clamp (|Z| <= 255) and
-// keeps the sum from overflowing.
+// clamp(rne(x * r) + Z, -128, 127), Z in [-128, 127]. The product is held to the integer
+// bounds [-128 - Z, 127 - Z] before it is rounded -- rounding is monotone,
+// so holding to integer bounds before or after it gives the same integer --
+// and then rounded to nearest, ties to even, by adding 1.5 * 2^23, which
+// leaves rne(y) in the low mantissa bits (|y| <= 255 here). The code is the
+// low byte of those bits plus Z - 0x4B400000. A NaN product is held to the
+// lower bound (fmaxf returns the non-NaN operand): code -128.
 __device__ __forceinline__ uint2 quant8_asym_sat(const uint4 &v, float r, int z) {
+  const float lo = static_cast<float>(-128 - z), hi = static_cast<float>(127 - z);
+  const int bias = z - 0x4B400000;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   int q[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    q[2 * i] = min(max(rne_held(__fmul_rn(bf16_lo(w[i]), r)) + z, -128), 127);
-    q[2 * i + 1] = min(max(rne_held(__fmul_rn(bf16_hi(w[i]), r)) + z, -128), 127);  // low bytes: the codes
+    q[2 * i] = __float_as_int(__fadd_rn(fminf(fmaxf(__fmul_rn(bf16_lo(w[i]), r), lo), hi), 12582912.0f)) + bias;
+    q[2 * i + 1] = __float_as_int(__fadd_rn(fminf(fmaxf(__fmul_rn(bf16_hi(w[i]), r), lo), hi), 12582912.0f)) + bias;
   }
   return make_uint2(low_bytes4(q[0], q[1], q[2], q[3]), low_bytes4(q[4], q[5], q[6], q[7]));
+}
+
+// Byte b (0..3) of w sign-extended to 32 bits: one prmt whose selector copies
+// byte b into the lowest byte and replicates its sign bit (selector nibble
+// with the high bit set) into the other three.
+template <int b>
+__device__ __forceinline__ int sext_byte(uint32_t w) {
+  constexpr uint32_t kSel = b | ((b | 8u) << 4) | ((b | 8u) << 8) | ((b | 8u) << 12);
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "n"(kSel));
+  return static_cast<int>(r);
+}
+
+// S * (q - Z) for the 16 codes of one uint4 (code j in byte j), Z in
+// [-128, 127]. q - Z is turned into fp32 without the conversion unit: the
+// sign-extended code plus 0x4B400000 - Z is the bit pattern of
+// 1.5 * 2^23 + (q - Z) (|q - Z| <= 255), from which 1.5 * 2^23 is subtracted
+// exactly. The product is the one rounding, as in S * float(q - Z).
+__device__ __forceinline__ void dequant16(const uint4 &v, float S, int z, float (&y)[16]) {
+  const int bias = 0x4B400000 - z;
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int q[4] = {sext_byte<0>(w[i]), sext_byte<1>(w[i]), sext_byte<2>(w[i]), sext_byte<3>(w[i])};
+#pragma unroll
+    for (int b = 0; b < 4; ++b) y[4 * i + b] = __fmul_rn(S, __fsub_rn(__int_as_float(q[b] + bias), 12582912.0f));
+  }
 }
 
 // Running per-halfword maximum of bf16 magnitudes (two values per word).

@@ -60,7 +60,7 @@ cudaError_t ensure_kernel_smem(int bytes, bool max_carveout) {
 }
 
 cudaError_t launch_quant_per_token(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
-                                   int8_t *Xq, float *S_x, cudaStream_t s);
+                                   int8_t *Xq, float *S_x, int num_sms, cudaStream_t s);
 // pdl = true: may start while the previous kernel runs. It lets its own
 // dependents (the decode GEMM) launch at once, then waits for the previous
 // kernel before reading or writing anything.

@@ -23,14 +23,14 @@ namespace w8a8 {
 // ------------------------------------------------------------ per token
 // G threads per row (32 = one warp, or 256 = the whole block), VPT 16-byte
 // chunks (8 bf16) per thread held in registers, so X is read exactly once.
-// Warp-per-row blocks hold 4 rows, so the rows spread evenly over the SMs.
-template <int G, int VPT>
+// Warp-per-row blocks hold RB rows (RB warps).
+template <int G, int VPT, int RB>
 __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__restrict__ X,
                                                               int64_t M, int64_t K, int64_t ldx,
                                                               int8_t *__restrict__ Xq,
                                                               float *__restrict__ S_x) {
-  constexpr int NT = G == 32 ? 128 : 256;  // threads per block
-  constexpr int R = NT / G;                // rows per block
+  constexpr int NT = G == 32 ? 32 * RB : 256;  // threads per block
+  constexpr int R = NT / G;                    // rows per block
   __shared__ uint32_t red[8];
   const int tid = threadIdx.x;
   const int g = tid / G;  // row slot in this block
@@ -82,10 +82,10 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__
   }
 }
 
-template <int G, int VPT>
+template <int G, int VPT, int RB = 4>
 static cudaError_t launch_per_token_t(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                       int8_t *Xq, float *S_x, cudaStream_t s) {
-  constexpr int NT = G == 32 ? 128 : 256;
+  constexpr int NT = G == 32 ? 32 * RB : 256;
   constexpr int R = NT / G;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((M + R - 1) / R));
@@ -96,17 +96,34 @@ static cudaError_t launch_per_token_t(const uint16_t *X, int64_t M, int64_t K, i
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quant_per_token_kernel<G, VPT>, X, M, K, ldx, Xq, S_x);
+  return cudaLaunchKernelEx(&cfg, quant_per_token_kernel<G, VPT, RB>, X, M, K, ldx, Xq, S_x);
+}
+
+// Rows (warps) per block of the warp-per-row form at 16 chunks per thread.
+// The block scheduler fills an SM up to its occupancy (about 22 of these
+// warps, by registers) before it moves on, so with small blocks some SMs take
+// far more rows than the average. Blocks of 8 rows allow at most 2 per SM, 16
+// rows, which is the even share when M is at most 2 x 8 rows per SM; with
+// more rows than that (two waves), blocks of 2 rows even out the second wave.
+static int per_token_rows_per_block(int64_t M, int num_sms) {
+  if (M >= static_cast<int64_t>(8) * num_sms && M <= static_cast<int64_t>(16) * num_sms) return 8;
+  return M > static_cast<int64_t>(16) * num_sms ? 2 : 4;
 }
 
 cudaError_t launch_quant_per_token(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
-                                   int8_t *Xq, float *S_x, cudaStream_t s) {
+                                   int8_t *Xq, float *S_x, int num_sms, cudaStream_t s) {
   const int64_t chunks = K / 8;
   if (chunks <= 32 * 1) return launch_per_token_t<32, 1>(X, M, K, ldx, Xq, S_x, s);
   if (chunks <= 32 * 2) return launch_per_token_t<32, 2>(X, M, K, ldx, Xq, S_x, s);
   if (chunks <= 32 * 4) return launch_per_token_t<32, 4>(X, M, K, ldx, Xq, S_x, s);
   if (chunks <= 32 * 8) return launch_per_token_t<32, 8>(X, M, K, ldx, Xq, S_x, s);
-  if (chunks <= 32 * 16) return launch_per_token_t<32, 16>(X, M, K, ldx, Xq, S_x, s);
+  if (chunks <= 32 * 16) {
+    switch (per_token_rows_per_block(M, num_sms)) {
+      case 8: return launch_per_token_t<32, 16, 8>(X, M, K, ldx, Xq, S_x, s);
+      case 2: return launch_per_token_t<32, 16, 2>(X, M, K, ldx, Xq, S_x, s);
+      default: return launch_per_token_t<32, 16, 4>(X, M, K, ldx, Xq, S_x, s);
+    }
+  }
   if (chunks <= 256 * 4) return launch_per_token_t<256, 4>(X, M, K, ldx, Xq, S_x, s);
   if (chunks <= 256 * 8) return launch_per_token_t<256, 8>(X, M, K, ldx, Xq, S_x, s);
   if (chunks <= 256 * 16) return launch_per_token_t<256, 16>(X, M, K, ldx, Xq, S_x, s);
@@ -192,13 +209,8 @@ __global__ void __launch_bounds__(256) dequant_per_tensor_kernel(const int8_t *_
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t m = i / cpr, c = i - m * cpr;
     const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(Xq + m * ldq) + c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     float y[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int q = static_cast<int8_t>((w[j >> 2] >> (8 * (j & 3))) & 0xFFu);
-      y[j] = __fmul_rn(S, __int2float_rn(q - z));
-    }
+    dequant16(v, S, z, y);
     if constexpr (BF16_OUT) {
       uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + m * K) + 2 * c;
       o[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),

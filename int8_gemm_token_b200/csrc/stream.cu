@@ -45,13 +45,8 @@ __device__ __forceinline__ void convert_piece(const uint4 &v, int64_t e, void *o
   if constexpr (C == Conv::kQuant) {  // 8 bf16 -> 8 codes
     *reinterpret_cast<uint2 *>(static_cast<int8_t *>(out) + e) = quant8_asym_sat(v, a, z);
   } else {  // 16 codes -> 16 values
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     float y[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int q = static_cast<int8_t>((w[j >> 2] >> (8 * (j & 3))) & 0xFFu);
-      y[j] = __fmul_rn(a, __int2float_rn(q - z));
-    }
+    dequant16(v, a, z, y);
     if constexpr (C == Conv::kDequantBf16) {
       uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + e);
       o[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
