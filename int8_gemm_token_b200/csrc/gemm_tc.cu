@@ -29,7 +29,9 @@
 //               quarter, the next 32 columns already in flight), the
 //               fixed-order fp32 dequant and bf16 / fp32 / int32 stores.
 //               The mixed (LLM.int8()) instantiation adds the 16-bit side
-//               product per element and keeps a serial per-chunk epilogue.
+//               product per element; in the CTA-pair kernel the tile's first
+//               16 outlier rows of W are staged in shared memory with the
+//               constants, so the side product reads no global memory.
 // Double-buffered accumulators let the epilogue of tile i overlap the MMAs
 // of tile i+1. Programmatic dependent launch: the first ring of weight tiles
 // is requested before griddepcontrol.wait, everything else after it. Every
@@ -48,6 +50,10 @@ constexpr int kBK = 128;              // bytes of K per stage = one 128B swizzle
 constexpr int kStageA = kBM * kBK;    // 16 KiB
 constexpr int kThreads = 256;
 constexpr int kEpiWarp0 = 4;
+// Mixed CTA-pair kernel: the first kSideRows outlier rows of W, for the
+// tile's 256 columns, are staged in shared memory per accumulator slot.
+constexpr int kSideRows = 16;
+constexpr int kSideStride = 256;  // staged row length (bf16 elements)
 
 template <int BN, int STAGES>
 struct TcConfig {
@@ -191,19 +197,40 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&acc)[32], int64_
 
 // The same fixed-order epilogue for 32 columns, with the per-column constants
 // already in shared memory (s_sw = s_w[n]; s_add = 0 + bias[n] without the
-// side path, bias[n] with it; s_cs = colsum[n]; zeros past N).
+// side path, bias[n] with it; s_cs = colsum[n]; zeros past N). With the side
+// path, outliers j < ns come from the staged rows s_wo (row j at
+// j * kSideStride, zeros past N) and this row's Xo values packed two per word
+// in xo2; outliers ns .. nuse-1 are read from W in global memory. The chain
+// runs over j in ascending order either way.
 template <bool MIXED>
 __device__ __forceinline__ void epilogue_chunk_s(const uint32_t (&acc)[32], int64_t m, int64_t n0, int64_t M,
                                                  int64_t N, float sx, int32_t z, const EpilogueArgs &ep,
                                                  int32_t nuse, const float *s_sw, const float *s_add,
-                                                 const int32_t *s_cs) {
+                                                 const int32_t *s_cs, const uint16_t *s_wo,
+                                                 const uint32_t (&xo2)[kSideRows / 2], int32_t ns) {
   if (m >= M) return;
   const bool full = n0 + 32 <= N;
   float side[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) side[i] = 0.0f;
   if (MIXED) {
-    for (int32_t j = 0; j < nuse; ++j) {
+#pragma unroll
+    for (int j = 0; j < kSideRows; ++j) {
+      if (j < ns) {
+        const float xo = (j & 1) ? bf16_hi(xo2[j >> 1]) : bf16_lo(xo2[j >> 1]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(s_wo + j * kSideStride + 8 * i);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            side[8 * i + 2 * h] = __fmaf_rn(xo, bf16_lo(w4[h]), side[8 * i + 2 * h]);
+            side[8 * i + 2 * h + 1] = __fmaf_rn(xo, bf16_hi(w4[h]), side[8 * i + 2 * h + 1]);
+          }
+        }
+      }
+    }
+    for (int32_t j = ns; j < nuse; ++j) {
       const float xo = __uint_as_float(static_cast<uint32_t>(ep.Xo[m * ep.cap + j]) << 16);
       const uint16_t *wrow = ep.W + static_cast<int64_t>(__ldg(ep.outlier_idx + j)) * ep.ldw + n0;
       if (full && (ep.ldw % 8) == 0) {
@@ -511,6 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           epilogue_chunk<MIXED>(r, m, nbase + c * 32, M, N, sx, z, ep, nuse);
         }
       } else {
+        const uint32_t kNoSide[kSideRows / 2] = {};
         uint32_t ra[32], rb[32];
         tmem_ld_32x32b_x32(taddr, ra);
 #pragma unroll
@@ -518,11 +546,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();  // chunk c in ra
           tmem_ld_32x32b_x32(taddr + (c + 1) * 32, rb);
           epilogue_chunk_s<MIXED>(ra, m, nbase + c * 32, M, N, sx, z, ep, nuse, c_sw + c * 32, c_add + c * 32,
-                                  c_cs + c * 32);
+                                  c_cs + c * 32, nullptr, kNoSide, 0);
           tmem_ld_wait();  // chunk c + 1 in rb
           if (c + 2 < BN / 32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, ra);
           epilogue_chunk_s<MIXED>(rb, m, nbase + (c + 1) * 32, M, N, sx, z, ep, nuse, c_sw + (c + 1) * 32,
-                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32);
+                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32, nullptr, kNoSide, 0);
         }
       }
       tc_fence_before();
@@ -574,7 +602,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // per-column epilogue constants of the tile, one slot per accumulator:
   // [slot][s_w | add | colsum][kTileN]
   float *sConst = reinterpret_cast<float *>(sB + STAGES * kStageB2);
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sConst + 2 * 3 * kTileN);
+  // mixed: the tile's first kSideRows outlier rows of W, one slot per
+  // accumulator: [slot][row][kTileN] bf16
+  constexpr int kSideElems = MIXED ? 2 * kSideRows * kTileN : 0;
+  static_assert(kTileN == kSideStride, "staged side rows are one tile wide");
+  uint16_t *sSide = reinterpret_cast<uint16_t *>(sConst + 2 * 3 * kTileN);
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sSide + kSideElems);
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *tfull_bar = empty_bar + STAGES;
   uint64_t *tempty_bar = tfull_bar + 2;
@@ -704,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float *c_sw = sConst + acc * 3 * kTileN, *c_add = c_sw + kTileN;
       int32_t *c_cs = reinterpret_cast<int32_t *>(c_add + kTileN);
 #pragma unroll
-      for (int j = 0; j < (MIXED ? 0 : 2); ++j) {
+      for (int j = 0; j < 2; ++j) {
         const int col = q * 64 + j * 32 + lane;
         const int64_t n = nbase + col;
         float sw = 0.0f, add = 0.0f;
@@ -717,6 +750,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         c_sw[col] = sw;
         c_add[col] = add;
         c_cs[col] = cs;
+      }
+      const int64_t m = (tile % num_m) * kTileM + rank * kHalf + q * 32 + lane;
+      uint16_t *c_wo = sSide + acc * kSideRows * kTileN;
+      int32_t ns = 0;
+      uint32_t xo2[kSideRows / 2];
+#pragma unroll
+      for (int j = 0; j < kSideRows / 2; ++j) xo2[j] = 0;
+      if constexpr (MIXED) {
+        // the side inputs of this tile, while its MMAs run: warp q stages
+        // outlier rows q, q + 4, ... of W (lane: 8 columns); every thread
+        // keeps its own row's Xo values
+        ns = nuse < kSideRows ? nuse : kSideRows;
+        for (int j = q; j < ns; j += 4) {
+          const uint16_t *wrow = ep.W + static_cast<int64_t>(__ldg(ep.outlier_idx + j)) * ep.ldw + nbase;
+          const int col = lane * 8;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if ((ep.ldw % 8) == 0 && nbase + col + 8 <= N) {
+            v = __ldg(reinterpret_cast<const uint4 *>(wrow + col));
+          } else {
+            uint32_t e[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) e[t] = nbase + col + t < N ? __ldg(wrow + col + t) : 0u;
+            v = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
+          }
+          *reinterpret_cast<uint4 *>(c_wo + j * kTileN + col) = v;
+        }
+        if (m < M) {
+          const uint16_t *xrow = ep.Xo + m * ep.cap;
+#pragma unroll
+          for (int j = 0; j < kSideRows; ++j)
+            if (j < ns) xo2[j >> 1] |= static_cast<uint32_t>(__ldg(xrow + j)) << (16 * (j & 1));
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&cready_bar[acc]);
@@ -731,21 +796,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int64_t m = (tile % num_m) * kTileM + rank * kHalf + q * 32 + lane;
       float sx = 0.0f;
       if (m < M) sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : __ldg(ep.S_x);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kTileN);
-      if constexpr (MIXED) {
-        // the side path's epilogue is long: one chunk at a time, constants
-        // read per chunk (measured faster here than the staged form)
-#pragma unroll 1
-        for (int c = 0; c < kTileN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + c * 32, r);
-          tmem_ld_wait();
-          epilogue_chunk<MIXED>(r, m, nbase + c * 32, M, N, sx, z, ep, nuse);
-        }
-      } else {
+      {
         uint32_t ra[32], rb[32];
         tmem_ld_32x32b_x32(taddr, ra);
 #pragma unroll
@@ -753,11 +807,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();  // chunk c in ra
           tmem_ld_32x32b_x32(taddr + (c + 1) * 32, rb);
           epilogue_chunk_s<MIXED>(ra, m, nbase + c * 32, M, N, sx, z, ep, nuse, c_sw + c * 32, c_add + c * 32,
-                                  c_cs + c * 32);
+                                  c_cs + c * 32, c_wo + c * 32, xo2, ns);
           tmem_ld_wait();  // chunk c + 1 in rb
           if (c + 2 < kTileN / 32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, ra);
           epilogue_chunk_s<MIXED>(rb, m, nbase + (c + 1) * 32, M, N, sx, z, ep, nuse, c_sw + (c + 1) * 32,
-                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32);
+                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32, c_wo + (c + 1) * 32, xo2, ns);
         }
       }
       tc_fence_before();
@@ -788,8 +842,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int STAGES, bool MIXED>
 cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                          const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
-  // ring + epilogue constants + 1 KiB alignment slack + barriers and flags (< 256 B)
-  constexpr size_t kSmem = static_cast<size_t>(STAGES) * 2 * 128 * kBK + 2 * 3 * 256 * 4 + 1024 + 256;
+  // ring + epilogue constants (+ staged side rows) + 1 KiB alignment slack +
+  // barriers and flags (< 256 B)
+  constexpr size_t kSmem = static_cast<size_t>(STAGES) * 2 * 128 * kBK + 2 * 3 * 256 * 4 +
+                           (MIXED ? 2 * kSideRows * 256 * 2 : 0) + 1024 + 256;
   static_assert((2 * STAGES + 7) * 8 + 4 * 4 <= 256, "barriers and flags fit their reserve");
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   alignas(64) CUtensorMap tmA, tmB;

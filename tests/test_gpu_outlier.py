@@ -80,13 +80,17 @@ def test_outlier_split_thresholds_and_overflow():
 @pytest.mark.parametrize("M,K,N,cols", [(16, 256, 512, [3, 200]), (300, 400, 520, [0, 399]),
                                         (129, 1024, 257, [17, 18, 19, 700, 1000, 1023]), (5, 128, 128, []),
                                         (32, 4096, 4096, [1, 2000, 4000]),
-                                        (520, 400, 5400, [5, 6, 390])])
+                                        (520, 400, 5400, [5, 6, 390]),
+                                        # CTA-pair tiles past the 16 staged outlier rows: an odd N (row
+                                        # stride not a multiple of 8 elements) and 17 at a ragged N
+                                        (300, 1024, 1001, list(range(3, 1000, 50))),
+                                        (260, 512, 520, [7 * i + 1 for i in range(17)])])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_mixed_decomp_gemm_bit_exact(M, K, N, cols, out_dtype):
     X = planted(M, K, cols, seed=3 * M + K)
     Wb = synth.bf16_bits(synth.weight(np.random.default_rng(N + K), K, N))
     bias = synth.bias(np.random.default_rng(5), N)
-    cap = 16
+    cap = 16 if len(cols) <= 16 else 32
     Wd = dev_bf16(Wb)
     Wq, s_w, _ = W.w8a8_quant_weight_per_channel(Wd)
     Xq, S_x, idx, n_out, Xo = W.int8_outlier_split(dev_bf16(X), 6.0, cap)
