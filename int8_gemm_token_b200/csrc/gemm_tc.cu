@@ -195,6 +195,43 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&acc)[32], int64_
   }
 }
 
+// Staged bf16 output of the CTA-pair kernel: each epilogue warp owns 32 rows x
+// 128 bytes of shared memory, laid out as the SWIZZLE_128B box of the output
+// tensor map (the 16-byte chunk c of row r at chunk c ^ (r % 8)); two 32-column
+// chunks fill it, then one TMA store writes the 32 x 64 block.
+constexpr int kStageBytes = 32 * 128;
+
+// This lane's 32 results as bf16 into half `half` (64 bytes) of its row.
+__device__ __forceinline__ void stage_bf16_row32(const float (&y)[32], uint8_t *stage, int lane, int half) {
+  uint8_t *row = stage + lane * 128;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int cc = 4 * half + c;
+    *reinterpret_cast<uint4 *>(row + ((cc ^ (lane & 7)) << 4)) =
+        make_uint4(pack_bf16x2(y[8 * c], y[8 * c + 1]), pack_bf16x2(y[8 * c + 2], y[8 * c + 3]),
+                   pack_bf16x2(y[8 * c + 4], y[8 * c + 5]), pack_bf16x2(y[8 * c + 6], y[8 * c + 7]));
+  }
+}
+
+// The warp's staged block to out[y .. y+32, x .. x+64) with one TMA store
+// (rows and columns past the tensor's end are clipped by the copy).
+__device__ __forceinline__ void flush_stage_bf16(const CUtensorMap *tmOut, uint8_t *stage, int lane, int64_t x,
+                                                 int64_t y) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmOut, stage, static_cast<int32_t>(x), static_cast<int32_t>(y));
+    bulk_commit_group();
+  }
+}
+
+// Before the staging rows are written again: the warp's previous TMA store
+// has finished reading them.
+__device__ __forceinline__ void stage_bf16_free(int lane) {
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+}
+
 // The same fixed-order epilogue for 32 columns, with the per-column constants
 // already in shared memory (s_sw = s_w[n]; s_add = 0 + bias[n] without the
 // side path, bias[n] with it; s_cs = colsum[n]; zeros past N). With the side
@@ -207,7 +244,8 @@ __device__ __forceinline__ void epilogue_chunk_s(const uint32_t (&acc)[32], int6
                                                  int64_t N, float sx, int32_t z, const EpilogueArgs &ep,
                                                  int32_t nuse, const float *s_sw, const float *s_add,
                                                  const int32_t *s_cs, const uint16_t *s_wo,
-                                                 const uint32_t (&xo2)[kSideRows / 2], int32_t ns) {
+                                                 const uint32_t (&xo2)[kSideRows / 2], int32_t ns,
+                                                 uint8_t *stage = nullptr, int half = 0) {
   if (m >= M) return;
   const bool full = n0 + 32 <= N;
   float side[32];
@@ -274,6 +312,10 @@ __device__ __forceinline__ void epilogue_chunk_s(const uint32_t (&acc)[32], int6
       if (MIXED) add = ep.bias ? __fadd_rn(side[i + h], add) : side[i + h];
       y[i + h] = __fmaf_rn(__int2float_rn(c), __fmul_rn(sx, sw4[h]), add);
     }
+  }
+  if (stage) {  // bf16 into this lane's staging row, for the warp's TMA store
+    stage_bf16_row32(y, stage, threadIdx.x & 31, half);
+    return;
   }
   if (ep.out_dtype == W8A8_BF16) {
     uint16_t *o = static_cast<uint16_t *>(ep.out) + m * N + n0;
@@ -587,8 +629,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int STAGES, bool MIXED>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       int64_t M, int64_t N, int64_t K, const __grid_constant__ EpilogueArgs ep,
-                       int32_t *status, uint64_t limit_ns) {
+                       const __grid_constant__ CUtensorMap tmOut, int32_t tma_store, int64_t M, int64_t N,
+                       int64_t K, const __grid_constant__ EpilogueArgs ep, int32_t *status, uint64_t limit_ns) {
   constexpr int kHalf = 128;                 // rows of A and of B per CTA
   constexpr int kStageA2 = kHalf * kBK;      // 16 KiB
   constexpr int kStageB2 = kHalf * kBK;      // 16 KiB
@@ -607,7 +649,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kSideElems = MIXED ? 2 * kSideRows * kTileN : 0;
   static_assert(kTileN == kSideStride, "staged side rows are one tile wide");
   uint16_t *sSide = reinterpret_cast<uint16_t *>(sConst + 2 * 3 * kTileN);
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sSide + kSideElems);
+  // plain: each epilogue warp's bf16 staging block for TMA stores (1 KiB aligned)
+  constexpr int kStageAll = MIXED ? 0 : 4 * kStageBytes;
+  uint8_t *sStage = reinterpret_cast<uint8_t *>(sSide + kSideElems);
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sStage + kStageAll);
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *tfull_bar = empty_bar + STAGES;
   uint64_t *tempty_bar = tfull_bar + 2;
@@ -799,6 +844,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sx = 0.0f;
       if (m < M) sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : __ldg(ep.S_x);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kTileN);
+      // bf16 output through this warp's staging block and TMA stores (32 rows x 64 columns each)
+      uint8_t *stg = (!MIXED && tma_store) ? sStage + q * kStageBytes : nullptr;
+      const int64_t mrow0 = (tile % num_m) * kTileM + rank * kHalf + q * 32;
       {
         uint32_t ra[32], rb[32];
         tmem_ld_32x32b_x32(taddr, ra);
@@ -806,12 +854,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kTileN / 32; c += 2) {
           tmem_ld_wait();  // chunk c in ra
           tmem_ld_32x32b_x32(taddr + (c + 1) * 32, rb);
+          if (stg) stage_bf16_free(lane);
           epilogue_chunk_s<MIXED>(ra, m, nbase + c * 32, M, N, sx, z, ep, nuse, c_sw + c * 32, c_add + c * 32,
-                                  c_cs + c * 32, c_wo + c * 32, xo2, ns);
+                                  c_cs + c * 32, c_wo + c * 32, xo2, ns, stg, 0);
           tmem_ld_wait();  // chunk c + 1 in rb
           if (c + 2 < kTileN / 32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, ra);
           epilogue_chunk_s<MIXED>(rb, m, nbase + (c + 1) * 32, M, N, sx, z, ep, nuse, c_sw + (c + 1) * 32,
-                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32, c_wo + (c + 1) * 32, xo2, ns);
+                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32, c_wo + (c + 1) * 32, xo2, ns, stg, 1);
+          if (stg && nbase + c * 32 < N && mrow0 < M) flush_stage_bf16(&tmOut, stg, lane, nbase + c * 32, mrow0);
         }
       }
       tc_fence_before();
@@ -826,6 +876,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc = 0;
         acc_phase ^= 1u;
       }
+    }
+    if (!MIXED && tma_store) {
+      if (lane == 0) bulk_wait_all();  // every store of this warp has completed before the CTA leaves
+      __syncwarp();
     }
   }
 
@@ -842,10 +896,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int STAGES, bool MIXED>
 cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                          const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
-  // ring + epilogue constants (+ staged side rows) + 1 KiB alignment slack +
-  // barriers and flags (< 256 B)
+  // ring + epilogue constants (+ staged side rows, or the epilogue warps'
+  // staging blocks) + 1 KiB alignment slack + barriers and flags (< 256 B)
   constexpr size_t kSmem = static_cast<size_t>(STAGES) * 2 * 128 * kBK + 2 * 3 * 256 * 4 +
-                           (MIXED ? 2 * kSideRows * 256 * 2 : 0) + 1024 + 256;
+                           (MIXED ? 2 * kSideRows * 256 * 2 : 4 * kStageBytes) + 1024 + 256;
   static_assert((2 * STAGES + 7) * 8 + 4 * 4 <= 256, "barriers and flags fit their reserve");
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   alignas(64) CUtensorMap tmA, tmB;
@@ -855,6 +909,16 @@ cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t 
   if (!encode_tmap_2d(&tmB, Wq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                       static_cast<uint64_t>(K), kBK, 128, true))
     return cudaErrorInvalidValue;
+  // bf16 output rows that are whole 16-byte multiples go out through TMA stores
+  const int32_t tma_store = !MIXED && ep.out_dtype == W8A8_BF16 && (N % 8) == 0;
+  alignas(64) CUtensorMap tmOut;
+  if (tma_store) {
+    if (!encode_tmap_2d(&tmOut, ep.out, TmapType::kBF16, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                        static_cast<uint64_t>(N) * 2, 64, 32, true))
+      return cudaErrorInvalidValue;
+  } else {
+    tmOut = tmA;  // never used: the epilogue stores directly
+  }
   auto kern = gemm_i8_tc2_kernel<STAGES, MIXED>;
   cudaError_t e = ensure_kernel_smem<gemm_i8_tc2_kernel<STAGES, MIXED>>(static_cast<int>(kSmem), false);
   if (e != cudaSuccess) return e;
@@ -874,7 +938,7 @@ cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, M, N, K, ep, status, kWaitLimitNs);
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmOut, tma_store, M, N, K, ep, status, kWaitLimitNs);
 }
 
 template <int BN, int STAGES, bool MIXED>
