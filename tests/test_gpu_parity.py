@@ -122,7 +122,10 @@ def test_gemm_int32_accumulator_bit_exact(M, N, K):
 # does the same with ragged edges.
 @pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 400), (200, 264, 512), (520, 5000, 400),
                                    (520, 5400, 256), (520, 5800, 272), (200, 11008, 512), (100, 2000, 400),
-                                   (2048, 20480, 512), (1000, 18000, 208)])
+                                   (2048, 20480, 512), (1000, 18000, 208),
+                                   # CTA-pair tiles: rows of bf16 output that are not 16-byte multiples
+                                   # (direct stores), and one tile whose only valid 64-column box is partial
+                                   (260, 1001, 272), (300, 40, 128)])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_prefill_linear_bit_exact(M, N, K, out_dtype):
     X, Wf, b = _rand_case(M, N, K, 3 * M + N)
