@@ -27,11 +27,15 @@
 //               colsum) staged in shared memory while its MMAs run, then
 //               tcgen05.ld of the int32 accumulator (each warp its 32-lane
 //               quarter, the next 32 columns already in flight), the
-//               fixed-order fp32 dequant and bf16 / fp32 / int32 stores.
+//               fixed-order fp32 dequant and bf16 / fp32 / int32 stores
+//               (in the CTA-pair kernel, bf16 rows that are whole 16-byte
+//               multiples go through a per-warp shared-memory block and TMA
+//               tensor stores).
 //               The mixed (LLM.int8()) instantiation adds the 16-bit side
 //               product per element; in the CTA-pair kernel the tile's first
 //               16 outlier rows of W are staged in shared memory with the
-//               constants, so the side product reads no global memory.
+//               constants, so up to 16 outliers the side product reads no
+//               global memory.
 // Double-buffered accumulators let the epilogue of tile i overlap the MMAs
 // of tile i+1. Programmatic dependent launch: the first ring of weight tiles
 // is requested before griddepcontrol.wait, everything else after it. Every
