@@ -12,8 +12,13 @@
 // Pass 1 (column flags): each thread owns 8 adjacent columns (one 16-byte
 //   load per row) over a band of 16 rows, with all 16 loads in flight at
 //   once, keeps the largest magnitude per column and sets the columns' bits
-//   in a K-bit workspace bitmap when it exceeds the threshold (atomicOr only for outlier columns, so almost never). X is
-//   loaded under an L2 evict-last policy so that pass 2 finds it in L2.
+//   in a K-bit workspace bitmap when it exceeds the threshold (atomicOr only
+//   for outlier columns, so almost never). X is loaded under an L2
+//   evict-last policy, so that pass 2 finds it in L2. The bitmap is cleared
+//   by a one-block kernel just before pass 1; both launch with programmatic
+//   dependent launch, so pass 1 streams X while the bitmap is cleared and
+//   waits for the clearing only before its first flag (a memset between
+//   them cost about 3 us per call).
 // Pass 2 (rows): a grid sized to fill the SMs once; every CTA turns the
 //   bitmap into the ascending index list (block-wide popcount scan) and
 //   copies the bitmap into shared memory once; CTA 0 publishes the list and
@@ -90,7 +95,20 @@ __global__ void __launch_bounds__(256) outlier_colflag_kernel(const uint16_t *__
     if (__uint_as_float(mw[j] << 16) > threshold) bits |= 1u << (2 * j);
     if (__uint_as_float(mw[j] & 0xFFFF0000u) > threshold) bits |= 2u << (2 * j);
   }
+  // the bitmap is cleared by the kernel before this one: wait for it before the first flag
+  pdl_wait_prerequisite();
   if (bits) atomicOr(bitmap + ((g * 8) >> 5), bits << ((g * 8) & 31));
+}
+
+// Clears the column bitmap for pass 1. Launched with programmatic dependent
+// launch: it waits for the previous kernel (the row pass of a previous split
+// may still read the bitmap), then lets pass 1 launch -- the input X is final
+// by then, so pass 1 streams it at once and waits for this kernel only before
+// its first flag -- and then clears the words.
+__global__ void __launch_bounds__(256) outlier_clear_kernel(uint32_t *__restrict__ bitmap, int64_t words) {
+  pdl_wait_prerequisite();
+  pdl_launch_dependents();
+  for (int64_t w = threadIdx.x; w < words; w += blockDim.x) bitmap[w] = 0u;
 }
 
 // ------------------------------------------------------------------ pass 2
@@ -291,12 +309,25 @@ cudaError_t launch_outlier_split(const uint16_t *X, int64_t M, int64_t K, int64_
                                  int8_t *Xq, float *S_x, int32_t *idx, int32_t *n_out, uint16_t *Xo, void *workspace,
                                  int num_sms, int32_t *status, cudaStream_t s) {
   uint32_t *bitmap = static_cast<uint32_t *>(workspace);
-  cudaError_t e = cudaMemsetAsync(bitmap, 0, outlier_workspace_bytes(K), s);
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t c0 = {};
+  c0.gridDim = dim3(1);
+  c0.blockDim = dim3(256);
+  c0.stream = s;
+  c0.attrs = pdl;
+  c0.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&c0, outlier_clear_kernel, bitmap, static_cast<int64_t>((K + 31) / 32));
   if (e != cudaSuccess) return e;
   const int64_t groups = K / 8;
-  const dim3 grid1(static_cast<unsigned>((groups + 255) / 256), static_cast<unsigned>((M + kRowsPerThread - 1) / kRowsPerThread));
-  outlier_colflag_kernel<<<grid1, 256, 0, s>>>(X, M, K, ldx, threshold, bitmap);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t c1 = {};
+  c1.gridDim = dim3(static_cast<unsigned>((groups + 255) / 256), static_cast<unsigned>((M + kRowsPerThread - 1) / kRowsPerThread));
+  c1.blockDim = dim3(256);
+  c1.stream = s;
+  c1.attrs = pdl;
+  c1.numAttrs = 1;
+  e = cudaLaunchKernelEx(&c1, outlier_colflag_kernel, X, M, K, ldx, threshold, bitmap);
   if (e != cudaSuccess) return e;
   const int64_t chunks = K / 8;
   if (chunks <= 32 * 4) return launch_rows_t<32, 4>(X, M, K, ldx, bitmap, cap, Xq, S_x, idx, n_out, Xo, num_sms, status, s);
