@@ -60,6 +60,28 @@ def test_outlier_split_bit_exact(M, K, cols, ld_pad):
     assert n >= len(cols) and st == 0
 
 
+@pytest.mark.parametrize("M,K", [(300, 4112), (4096, 8192), (7, 24576)])
+def test_outlier_split_reuses_a_dirty_workspace(M, K):
+    """The call clears its column bitmap itself: a workspace filled with ones,
+    then two back-to-back splits with different outlier columns on that same
+    workspace (the second launched while the first may still run), each equal
+    to the oracle -- no flag may leak from the garbage or from the first call."""
+    cols_a, cols_b = [0, 33, K - 1], [5, K // 2 + 1]
+    Xa = planted(M, K, cols_a, seed=M + 1, clip=5.5)
+    Xb = planted(M, K, cols_b, seed=M + 2, clip=5.5)
+    cap = 8
+    ws = torch.full((int(W.lib().int8_outlier_split_workspace_size(K)),), 255, dtype=torch.uint8, device="cuda")
+    outs = [W.int8_outlier_split(dev_bf16(X), 6.0, cap, workspace=ws) for X in (Xa, Xb)]
+    assert W.w8a8_check_device_error() == 0
+    for X, cols, (Xq, S_x, idx, n_out, Xo) in zip((Xa, Xb), (cols_a, cols_b), outs):
+        rq, rS, ridx, rn, rXo = oracle.outlier_split(X, 6.0, cap)
+        assert rn == len(cols) and int(host(n_out)[0]) == rn
+        assert_same(host(idx)[:rn], ridx[:rn], "outlier_idx")
+        assert_same(host(Xq), rq, "Xq")
+        assert_same(host(S_x), rS, "S_x")
+        assert_same(host_bf16(Xo)[:, :rn], rXo[:, :rn], "Xo")
+
+
 def test_outlier_split_thresholds_and_overflow():
     X = planted(64, 512, [3, 70, 300], seed=1)
     n, st = check_split(X, float("inf"), 16)
