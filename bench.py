@@ -66,7 +66,7 @@ TC2_TRAFFIC = {
     "bytes": 53_672_448 + 10_807_552,
     "sources": ["int8_gemm_token_b200/csrc/gemm_tc.cu", "int8_gemm_token_b200/csrc/gemm_pair.cuh",
                 "int8_gemm_token_b200/csrc/device.cuh", "int8_gemm_token_b200/csrc/kernels.h"],
-    "sources_sha256": "f46426b09543625da75c913a515185a23569e0360dc6e809a6bf162ee8a098bc",
+    "sources_sha256": "25c1e814b4f0463842eb89125634fcf0994831116e22326a25adacb16a2fc6cc",
     "profile": "profiles/gemm_i8_tc2_prefill_7b_2048x4096x11008.txt",
 }
 

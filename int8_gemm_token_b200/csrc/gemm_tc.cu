@@ -32,10 +32,9 @@
 //               multiples go through a per-warp shared-memory block and TMA
 //               tensor stores).
 //               The mixed (LLM.int8()) instantiation adds the 16-bit side
-//               product per element; in the CTA-pair kernel the tile's first
-//               16 outlier rows of W are staged in shared memory with the
-//               constants, so up to 16 outliers the side product reads no
-//               global memory.
+//               product per element; the tile's first 16 outlier rows of W
+//               are staged in shared memory with the constants, so up to 16
+//               outliers the side product reads no global memory.
 // Double-buffered accumulators let the epilogue of tile i overlap the MMAs
 // of tile i+1. Programmatic dependent launch: the first ring of weight tiles
 // is requested before griddepcontrol.wait, everything else after it. Every
@@ -59,145 +58,19 @@ constexpr int kEpiWarp0 = 4;
 constexpr int kSideRows = 16;
 constexpr int kSideStride = 256;  // staged row length (bf16 elements)
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool MIXED = false>
 struct TcConfig {
   static constexpr int kStageB = BN * kBK;
   static constexpr int kTmemCols = 2 * BN;  // two accumulators
   static constexpr size_t kRing = static_cast<size_t>(STAGES) * (kStageA + kStageB);
-  static constexpr size_t kSmem = kRing + 2 * 3 * BN * 4 /*epilogue constants*/ + 1024 /*alignment slack*/ +
+  // mixed: the staged outlier rows of W, [slot][kSideRows][BN] bf16
+  static constexpr size_t kSide = MIXED ? static_cast<size_t>(2) * kSideRows * BN * 2 : 0;
+  static constexpr size_t kSmem = kRing + 2 * 3 * BN * 4 /*epilogue constants*/ + kSide + 1024 /*alignment slack*/ +
                                   256 /*barriers etc.*/;
+  static_assert(!MIXED || BN == kSideStride, "staged side rows are one tile wide");
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
 };
-
-// Fixed-order epilogue of one row segment of 32 columns (see include/w8a8.h):
-//   c = acc - Z*colsum[n]; y = fmaf(float(c), S_x*s_w[n], side + bias[n]).
-template <bool MIXED>
-__device__ __forceinline__ void epilogue_chunk(const uint32_t (&acc)[32], int64_t m, int64_t n0,
-                                               int64_t M, int64_t N, float sx, int32_t z,
-                                               const EpilogueArgs &ep, int32_t nuse) {
-  if (m >= M) return;
-  const bool full = n0 + 32 <= N;
-  float sw[32], bs[32];
-  int32_t cs[32];
-  if (full) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 v = __ldg(reinterpret_cast<const float4 *>(ep.s_w + n0) + i);
-      sw[4 * i] = v.x; sw[4 * i + 1] = v.y; sw[4 * i + 2] = v.z; sw[4 * i + 3] = v.w;
-    }
-    if (ep.bias) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(ep.bias + n0) + i);
-        bs[4 * i] = v.x; bs[4 * i + 1] = v.y; bs[4 * i + 2] = v.z; bs[4 * i + 3] = v.w;
-      }
-    }
-    if (z != 0) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int4 v = __ldg(reinterpret_cast<const int4 *>(ep.colsum + n0) + i);
-        cs[4 * i] = v.x; cs[4 * i + 1] = v.y; cs[4 * i + 2] = v.z; cs[4 * i + 3] = v.w;
-      }
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const bool ok = n0 + i < N;
-      sw[i] = ok ? __ldg(ep.s_w + n0 + i) : 0.0f;
-      bs[i] = (ok && ep.bias) ? __ldg(ep.bias + n0 + i) : 0.0f;
-      cs[i] = (ok && z != 0) ? __ldg(ep.colsum + n0 + i) : 0;
-    }
-  }
-
-  float side[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) side[i] = 0.0f;
-  if (MIXED) {
-    for (int32_t j = 0; j < nuse; ++j) {
-      const float xo = __uint_as_float(static_cast<uint32_t>(ep.Xo[m * ep.cap + j]) << 16);
-      const uint16_t *wrow = ep.W + static_cast<int64_t>(__ldg(ep.outlier_idx + j)) * ep.ldw + n0;
-      if (full && (ep.ldw % 8) == 0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4 *>(wrow) + i);
-          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            side[8 * i + 2 * h] = __fmaf_rn(xo, bf16_lo(w4[h]), side[8 * i + 2 * h]);
-            side[8 * i + 2 * h + 1] = __fmaf_rn(xo, bf16_hi(w4[h]), side[8 * i + 2 * h + 1]);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (n0 + i < N) {
-            const float wv = __uint_as_float(static_cast<uint32_t>(__ldg(wrow + i)) << 16);
-            side[i] = __fmaf_rn(xo, wv, side[i]);
-          }
-        }
-      }
-    }
-  }
-
-  float y[32];
-  int32_t craw[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    int32_t c = static_cast<int32_t>(acc[i]);
-    if (z != 0) c -= z * cs[i];
-    craw[i] = c;
-    const float f = __int2float_rn(c);
-    const float sc = __fmul_rn(sx, sw[i]);
-    float add = MIXED ? side[i] : 0.0f;
-    if (ep.bias) add = __fadd_rn(add, bs[i]);
-    y[i] = __fmaf_rn(f, sc, add);
-  }
-
-  if (ep.out_dtype == W8A8_BF16) {
-    uint16_t *o = static_cast<uint16_t *>(ep.out) + m * N + n0;
-    if (full && (N % 8) == 0) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint4 v;
-        v.x = pack_bf16x2(y[8 * i + 0], y[8 * i + 1]);
-        v.y = pack_bf16x2(y[8 * i + 2], y[8 * i + 3]);
-        v.z = pack_bf16x2(y[8 * i + 4], y[8 * i + 5]);
-        v.w = pack_bf16x2(y[8 * i + 6], y[8 * i + 7]);
-        reinterpret_cast<uint4 *>(o)[i] = v;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (n0 + i < N) {
-          __nv_bfloat16 b = __float2bfloat16_rn(y[i]);
-          o[i] = *reinterpret_cast<uint16_t *>(&b);
-        }
-    }
-  } else if (ep.out_dtype == W8A8_FP32) {
-    float *o = static_cast<float *>(ep.out) + m * N + n0;
-    if (full && (N % 4) == 0) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        reinterpret_cast<float4 *>(o)[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (n0 + i < N) o[i] = y[i];
-    }
-  } else {
-    int32_t *o = static_cast<int32_t *>(ep.out) + m * N + n0;
-    if (full && (N % 4) == 0) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        reinterpret_cast<int4 *>(o)[i] = make_int4(craw[4 * i], craw[4 * i + 1], craw[4 * i + 2], craw[4 * i + 3]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (n0 + i < N) o[i] = craw[i];
-    }
-  }
-}
 
 // Staged bf16 output of the CTA-pair kernel: each epilogue warp owns 32 rows x
 // 128 bytes of shared memory, laid out as the SWIZZLE_128B box of the output
@@ -236,13 +109,15 @@ __device__ __forceinline__ void stage_bf16_free(int lane) {
   __syncwarp();
 }
 
-// The same fixed-order epilogue for 32 columns, with the per-column constants
-// already in shared memory (s_sw = s_w[n]; s_add = 0 + bias[n] without the
-// side path, bias[n] with it; s_cs = colsum[n]; zeros past N). With the side
-// path, outliers j < ns come from the staged rows s_wo (row j at
-// j * kSideStride, zeros past N) and this row's Xo values packed two per word
-// in xo2; outliers ns .. nuse-1 are read from W in global memory. The chain
-// runs over j in ascending order either way.
+// Fixed-order epilogue of one row segment of 32 columns (see include/w8a8.h):
+//   c = acc - Z*colsum[n]; y = fmaf(float(c), S_x*s_w[n], side + bias[n]),
+// with the per-column constants already in shared memory (s_sw = s_w[n];
+// s_add = 0 + bias[n] without the side path, bias[n] with it;
+// s_cs = colsum[n]; zeros past N). With the side path, outliers j < ns come
+// from the staged rows s_wo (row j at j * kSideStride, zeros past N) and this
+// row's Xo values packed two per word in xo2; outliers ns .. nuse-1 are read
+// from W in global memory. The chain runs over j in ascending order either
+// way.
 template <bool MIXED>
 __device__ __forceinline__ void epilogue_chunk_s(const uint32_t (&acc)[32], int64_t m, int64_t n0, int64_t M,
                                                  int64_t N, float sx, int32_t z, const EpilogueArgs &ep,
@@ -371,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       int64_t M, int64_t N, int64_t K, const __grid_constant__ EpilogueArgs ep,
                       int32_t *status, uint64_t limit_ns) {
-  using Cfg = TcConfig<BN, STAGES>;
+  using Cfg = TcConfig<BN, STAGES, MIXED>;
   constexpr uint32_t kIdesc = idesc_i8(kBM, BN);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -380,7 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // per-column epilogue constants of the tile, one slot per accumulator:
   // [slot][s_w | add | colsum][BN]
   float *sConst = reinterpret_cast<float *>(base + Cfg::kRing);
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sConst + 2 * 3 * BN);
+  uint16_t *sSide = reinterpret_cast<uint16_t *>(sConst + 2 * 3 * BN);  // mixed: staged outlier rows of W
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sSide) + Cfg::kSide);
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *tfull_bar = empty_bar + STAGES;
   uint64_t *tempty_bar = tfull_bar + 2;
@@ -527,9 +403,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kEpiWarp0) {
     pdl_wait_prerequisite();  // S_x, scales, side inputs and `out` belong to the previous kernel until then
     // -------------------------------------------------- epilogue
-    // As in the CTA-pair kernel: the tile's per-column constants are staged in
-    // shared memory while its MMAs run, and (without the side path) the next
-    // chunk's tcgen05.ld is in flight while the current one is stored.
+    // As in the CTA-pair kernel: the tile's per-column constants (and, mixed,
+    // the first kSideRows outlier rows of W and this row's Xo values) are
+    // staged while its MMAs run, and the next chunk's tcgen05.ld is in flight
+    // while the current one is stored.
     const int q = warp - kEpiWarp0;  // TMEM lane quarter of this warp (warp % 4)
     const int32_t z = ep.Z ? __ldg(ep.Z) : 0;
     int32_t nuse = 0;
@@ -541,21 +418,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t nbase = (tile / num_m) * BN;
       float *c_sw = sConst + acc * 3 * BN, *c_add = c_sw + BN;
       int32_t *c_cs = reinterpret_cast<int32_t *>(c_add + BN);
-      if constexpr (!MIXED) {
 #pragma unroll
-        for (int j = 0; j < BN / 128; ++j) {
-          const int col = q * (BN / 4) + j * 32 + lane;
-          const int64_t n = nbase + col;
-          float sw = 0.0f, add = 0.0f;
-          int32_t cs = 0;
-          if (n < N) {
-            sw = __ldg(ep.s_w + n);
-            if (ep.bias) add = __fadd_rn(0.0f, __ldg(ep.bias + n));
-            if (z != 0) cs = __ldg(ep.colsum + n);
+      for (int j = 0; j < BN / 128; ++j) {
+        const int col = q * (BN / 4) + j * 32 + lane;
+        const int64_t n = nbase + col;
+        float sw = 0.0f, add = 0.0f;
+        int32_t cs = 0;
+        if (n < N) {
+          sw = __ldg(ep.s_w + n);
+          if (ep.bias) add = MIXED ? __ldg(ep.bias + n) : __fadd_rn(0.0f, __ldg(ep.bias + n));
+          if (z != 0) cs = __ldg(ep.colsum + n);
+        }
+        c_sw[col] = sw;
+        c_add[col] = add;
+        c_cs[col] = cs;
+      }
+      const int64_t m = (tile % num_m) * kBM + q * 32 + lane;
+      uint16_t *c_wo = sSide + (MIXED ? acc * kSideRows * BN : 0);
+      int32_t ns = 0;
+      uint32_t xo2[kSideRows / 2];
+#pragma unroll
+      for (int j = 0; j < kSideRows / 2; ++j) xo2[j] = 0;
+      if constexpr (MIXED) {
+        // warp q stages outlier rows q, q + 4, ... of W (lane: 8 columns)
+        ns = nuse < kSideRows ? nuse : kSideRows;
+        for (int j = q; j < ns; j += 4) {
+          const uint16_t *wrow = ep.W + static_cast<int64_t>(__ldg(ep.outlier_idx + j)) * ep.ldw + nbase;
+          const int col = lane * 8;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if ((ep.ldw % 8) == 0 && nbase + col + 8 <= N) {
+            v = __ldg(reinterpret_cast<const uint4 *>(wrow + col));
+          } else {
+            uint32_t e[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) e[t] = nbase + col + t < N ? __ldg(wrow + col + t) : 0u;
+            v = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
           }
-          c_sw[col] = sw;
-          c_add[col] = add;
-          c_cs[col] = cs;
+          *reinterpret_cast<uint4 *>(c_wo + j * BN + col) = v;
+        }
+        if (m < M) {
+          const uint16_t *xrow = ep.Xo + m * ep.cap;
+#pragma unroll
+          for (int j = 0; j < kSideRows; ++j)
+            if (j < ns) xo2[j >> 1] |= static_cast<uint32_t>(__ldg(xrow + j)) << (16 * (j & 1));
         }
       }
       __syncwarp();
@@ -571,20 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int64_t m = (tile % num_m) * kBM + q * 32 + lane;
       float sx = 0.0f;
       if (m < M) sx = ep.s_x_per_row ? __ldg(ep.S_x + m) : __ldg(ep.S_x);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      if constexpr (MIXED) {
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + c * 32, r);
-          tmem_ld_wait();
-          epilogue_chunk<MIXED>(r, m, nbase + c * 32, M, N, sx, z, ep, nuse);
-        }
-      } else {
-        const uint32_t kNoSide[kSideRows / 2] = {};
+      {
         uint32_t ra[32], rb[32];
         tmem_ld_32x32b_x32(taddr, ra);
 #pragma unroll
@@ -592,11 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();  // chunk c in ra
           tmem_ld_32x32b_x32(taddr + (c + 1) * 32, rb);
           epilogue_chunk_s<MIXED>(ra, m, nbase + c * 32, M, N, sx, z, ep, nuse, c_sw + c * 32, c_add + c * 32,
-                                  c_cs + c * 32, nullptr, kNoSide, 0);
+                                  c_cs + c * 32, c_wo + c * 32, xo2, ns);
           tmem_ld_wait();  // chunk c + 1 in rb
           if (c + 2 < BN / 32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, ra);
           epilogue_chunk_s<MIXED>(rb, m, nbase + (c + 1) * 32, M, N, sx, z, ep, nuse, c_sw + (c + 1) * 32,
-                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32, nullptr, kNoSide, 0);
+                                  c_add + (c + 1) * 32, c_cs + (c + 1) * 32, c_wo + (c + 1) * 32, xo2, ns);
         }
       }
       tc_fence_before();
@@ -948,7 +843,7 @@ cudaError_t launch_tc2_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t 
 template <int BN, int STAGES, bool MIXED>
 cudaError_t launch_tc_t(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
                         const EpilogueArgs &ep, int num_sms, int32_t *status, cudaStream_t s) {
-  using Cfg = TcConfig<BN, STAGES>;
+  using Cfg = TcConfig<BN, STAGES, MIXED>;
   alignas(64) CUtensorMap tmA, tmB;
   if (!encode_tmap_2d(&tmA, Xq, TmapType::kU8, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                       static_cast<uint64_t>(K), kBK, kBM, true))

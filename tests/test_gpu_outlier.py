@@ -106,7 +106,9 @@ def test_outlier_split_thresholds_and_overflow():
                                         # CTA-pair tiles past the 16 staged outlier rows: an odd N (row
                                         # stride not a multiple of 8 elements) and 17 at a ragged N
                                         (300, 1024, 1001, list(range(3, 1000, 50))),
-                                        (260, 512, 520, [7 * i + 1 for i in range(17)])])
+                                        (260, 512, 520, [7 * i + 1 for i in range(17)]),
+                                        # the same past 16 outliers in the single-CTA kernel (65..255 tokens)
+                                        (100, 1024, 1001, list(range(5, 1000, 50)))])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_mixed_decomp_gemm_bit_exact(M, K, N, cols, out_dtype):
     X = planted(M, K, cols, seed=3 * M + K)
