@@ -355,6 +355,11 @@ size_t int8_outlier_split_workspace_size(int64_t K);
  *   Wq, s_w   device, from w8a8_quant_weight_per_channel of W
  *   W         device bf16 [K, N], row stride ldw: the unquantized weight
  *   bias      device fp32 [N] or NULL;  out device [M, N], bf16 or fp32
+ * Cost: the side product runs on the CUDA cores, n_used fmaf per output
+ * element; the first 16 outlier rows of W are staged per tile in shared
+ * memory, later ones are read from global memory. This is the faster of the
+ * two mixed GEMMs up to 16 outlier columns; beyond that use
+ * int8_mixed_decomp_gemm_tc, whose cost barely grows with the count.
  */
 w8a8_status int8_mixed_decomp_gemm(const int8_t *Xq, const float *S_x, const void *Xo,
                                    const int32_t *outlier_idx, const int32_t *n_out, int32_t cap,
