@@ -214,6 +214,11 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
   for (int it = 0; grp < groups; grp += gridDim.x, ++it) {
     const int64_t m = grp * R + g;
     const bool row_ok = m < M;
+    // this row's first outlier value of this thread, requested now so that its
+    // round trip overlaps the reduction and quantization below
+    const uint16_t *xrow = X + m * ldx;
+    uint16_t xo_first = 0;
+    if (row_ok && t < nuse) xo_first = __ldg(xrow + s_dyn[t]);
     // next group's loads, in flight while this one is processed (when the
     // two rows fit in registers)
     constexpr bool kPrefetch = VPT <= 8;
@@ -259,9 +264,9 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
         const int64_t c = t + static_cast<int64_t>(j) * G;
         if (c < chunks) reinterpret_cast<uint2 *>(qrow)[c] = quant8_sym_sat(v[j], r);
       }
-      // gather this row's outlier values (the row is hot in L1/L2)
-      const uint16_t *xrow = X + m * ldx;
-      for (int j = t; j < nuse; j += G) Xo[m * cap + j] = __ldg(xrow + s_dyn[j]);
+      // this row's outlier values (the first one per thread loaded above)
+      if (t < nuse) Xo[m * cap + t] = xo_first;
+      for (int j = t + G; j < nuse; j += G) Xo[m * cap + j] = __ldg(xrow + s_dyn[j]);
     }
     if constexpr (kPrefetch) {
 #pragma unroll
