@@ -34,6 +34,7 @@
  * Readings where the pages are silent or garbled are marked "reading:".
  */
 #include <fenv.h>
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -78,8 +79,11 @@ int oracle_round_mode_ok(void) { return fegetround() == FE_TONEAREST; }
 
 /* round-half-even of an fp32 value, then clamped into [-1024, 1024] so that
  * the later integer add of a zero point cannot overflow; the final clamp to
- * the int8 range makes this pre-clamp invisible. */
+ * the int8 range makes this pre-clamp invisible. A NaN (0 * inf, possible
+ * only with an infinite r given to the static quantizer, which its contract
+ * excludes) is given code 0 here so that the C stays defined. */
 static int rne_clamped(float p) {
+    if (p != p) return 0;
     float t = nearbyintf(p);
     if (t < -1024.0f) t = -1024.0f;
     if (t > 1024.0f) t = 1024.0f;
@@ -95,6 +99,8 @@ static int clamp_int(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi 
 /* (configuration guide: prefill is per-token symmetric).                     */
 /* reading: scale by r = 127/a (one division per vector) rather than         */
 /* dividing each element by S; a == 0 gives S = r = 0 and all-zero codes.    */
+/* reading: so does an absmax so small (below 127/FLT_MAX, ~3.7e-37) that     */
+/* 127/a overflows fp32: no finite scale resolves such values on the grid.    */
 /* ------------------------------------------------------------------------ */
 static void absmax_quant_vector(const void *base, int dtype, int64_t start, int64_t stride,
                                 int64_t len, const unsigned char *skip, int8_t *q,
@@ -106,7 +112,7 @@ static void absmax_quant_vector(const void *base, int dtype, int64_t start, int6
         if (v > a) a = v;
     }
     float S = 0.0f, r = 0.0f;
-    if (a > 0.0f) {
+    if (a > 0.0f && 127.0f / a <= FLT_MAX) {
         S = a / 127.0f;
         r = 127.0f / a;
     }
@@ -168,13 +174,14 @@ void oracle_calibrate_static(const void *X, int dtype, int64_t T, int64_t K, int
             if (v > hi) hi = v;
         }
     }
-    if (hi == lo) {
+    float d = hi - lo;
+    if (hi == lo || !(255.0f / d <= FLT_MAX)) { /* reading: a range whose 255/d
+                                                 * overflows fp32 counts as empty */
         *S = 1.0f;
         *r = 1.0f;
         *Z = 0;
         return;
     }
-    float d = hi - lo;
     *S = d / 255.0f;
     *r = 255.0f / d;
     *Z = clamp_int(-128 - rne_clamped(lo * *r), -128, 127);

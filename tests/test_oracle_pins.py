@@ -93,6 +93,30 @@ def test_zero_row_gives_zero_scale_and_codes():
     assert np.all(Xq == 0) and np.all(S == 0)
 
 
+def test_tiny_vectors_quantize_as_zero():
+    """A row (or weight column) whose absmax a is below 127/FLT_MAX, where
+    127/a overflows fp32 (bf16 subnormals, tiny normals), is quantized as a
+    zero vector: S = 0 and all codes 0. Just above that bound the scale is
+    finite and the row's extreme values take codes +-127; a calibration range
+    whose 255/d overflows is treated like an empty one (S = r = 1, Z = 0)."""
+    fmax = float(np.finfo(np.float32).max)
+    tiny = np.array([1e-38, -1e-38, 3e-39, -9.2e-41, 0.0, -0.0, 2e-40, -5e-39], np.float32)
+    edge = np.array([4e-37, -4e-37, 1e-37, 0.0], np.float32)
+    X = bf(np.stack([tiny, tiny[::-1], np.zeros(8, np.float32), np.resize(edge, 8)]))
+    xf = f32(X)
+    a = np.abs(xf).max(axis=1)
+    assert np.all(a[:2] < 127.0 / fmax) and np.all(a[:2] > 0) and a[3] > 127.0 / fmax
+    Xq, S = oracle.quant_per_token(X)
+    assert np.all(Xq[:3] == 0) and np.all(S[:3] == 0)
+    assert S[3] > 0 and Xq[3, 0] == 127 and Xq[3, 1] == -127 and Xq[3, 3] == 0
+    Wq, s_w, colsum = oracle.quant_weight_per_channel(bf(np.stack([tiny, tiny[::-1]], axis=1)))
+    assert np.all(Wq == 0) and np.all(s_w == 0) and np.all(colsum == 0)
+    S, r, Z = oracle.calibrate_static(bf(tiny.reshape(2, 4)))
+    assert (S, r, Z) == (1.0, 1.0, 0)
+    S, r, Z = oracle.calibrate_static(bf(edge.reshape(1, 4) * 4))
+    assert 0 < r < fmax and -128 <= Z <= 127
+
+
 def test_weight_per_channel_pins():
     """One scale per output channel n over all K; colsum is the column sum of
     the int8 codes (numpy); round-trip bound per column."""
