@@ -74,7 +74,8 @@ const char *w8a8_status_string(w8a8_status status);
  * limitations paragraph (INT8 weights are re-quantized from 16-bit at load).
  *
  * For every output channel n: a = max_k |W[k, n]|, s_w[n] = a / 127,
- * Wq[n, k] = clamp(rne(W[k, n] * (127 / a)), -127, 127) (0 when a == 0), and
+ * Wq[n, k] = clamp(rne(W[k, n] * (127 / a)), -127, 127) (0, with s_w[n] = 0, when a == 0 or
+ * when 127 / a overflows fp32, a below 127/FLT_MAX ~ 3.7e-37), and
  * colsum[n] = sum_k Wq[n, k] (used by the zero-point correction).
  *   W       device, [K, N] row-major, row stride ldw elements; bf16 or fp32 (w_dtype)
  *   Wq      device, [N, K] int8, dense (row stride K), written
@@ -96,7 +97,8 @@ w8a8_status w8a8_quant_weight_per_channel(const void *W, w8a8_dtype w_dtype, int
  * Reading of the pages: the observed range is widened to contain 0,
  * lo = min(0, min X), hi = max(0, max X); then S = (hi - lo) / 255,
  * r = 255 / (hi - lo), Z = clamp(-128 - rne(lo * r), -128, 127); an all-zero
- * input gives S = r = 1, Z = 0.
+ * input, or a range so small that 255 / (hi - lo) overflows fp32, gives
+ * S = r = 1, Z = 0, so r is always finite.
  *   Xcal  device, [T, K] row-major, row stride ldx; bf16 or fp32 (x_dtype)
  *   S, r  device, one fp32 each, written;  Z  device, one int32, written
  * K here is any positive count (no multiple-of-16 rule). T*K must be > 0.
@@ -110,7 +112,9 @@ w8a8_status w8a8_calibrate_static(const void *Xcal, w8a8_dtype x_dtype, int64_t 
  * token); PDMIX configuration guide §3 (Prefill uses per-token symmetric
  * quantization, so Z_token = 0); LLM.int8() summary §一.1 absmax equation.
  * For each row m: a = max_k |X[m, k]|, S_x[m] = a / 127,
- * Xq[m, k] = clamp(rne(X[m, k] * (127 / a)), -127, 127) (0 when a == 0).
+ * Xq[m, k] = clamp(rne(X[m, k] * (127 / a)), -127, 127); a row with a == 0, or
+ * with a so small that 127 / a overflows fp32 (a below 127/FLT_MAX ~ 3.7e-37),
+ * is quantized as zero: S_x[m] = 0 and all codes 0.
  *   X    device bf16 [M, K], row stride ldx (>= K, multiple of 8)
  *   Xq   device int8 [M, K], dense, written
  *   S_x  device fp32 [M], written
@@ -126,7 +130,8 @@ w8a8_status w8a8_quant_per_token(const void *X, int64_t M, int64_t K, int64_t ld
  * w8a8_calibrate_static (device scalars, read by the kernel). Z is an int8
  * zero point, in [-128, 127] as w8a8_calibrate_static writes it; the result
  * for a Z outside that range is unspecified (the kernel cannot check a
- * device scalar without a synchronisation).
+ * device scalar without a synchronisation). r is finite (w8a8_calibrate_static
+ * never writes an infinite one); for an infinite r the codes are unspecified.
  *   X   device bf16 [M, K], row stride ldx;  Xq device int8 [M, K] dense, written
  */
 w8a8_status w8a8_quant_per_tensor(const void *X, int64_t M, int64_t K, int64_t ldx, const float *r,
@@ -320,6 +325,8 @@ w8a8_status w8a8_linear_static_noalloc(const void *X, int64_t M, int64_t K, int6
  *   X            device bf16 [M, K], row stride ldx
  *   Xq           device int8 [M, K] dense, written (outlier columns = 0)
  *   S_x          device fp32 [M], written: absmax over normal columns / 127
+ *                (0, with all of the row's codes 0, where that absmax is 0 or
+ *                so small that 127 / absmax overflows fp32)
  *   outlier_idx  device int32 [cap], written: first min(n, cap) indices
  *   n_out        device int32 scalar, written: the number n of outlier columns
  *   Xo           device bf16 [M, cap] dense, written: Xo[m, j] = X[m, idx[j]]

@@ -453,6 +453,19 @@ __device__ __forceinline__ uint2 quant8_sym_sat(const uint4 &v, float r) {
   return make_uint2(pack_sat_s8x4(q[0], q[1], q[2], q[3]), pack_sat_s8x4(q[4], q[5], q[6], q[7]));
 }
 
+// r = 127/a for a vector with absmax a, or 0 for a vector quantized as zero:
+// a = 0 (or NaN), or a so small (below 127/FLT_MAX, about 3.7e-37) that 127/a
+// overflows fp32 -- no finite scale resolves such values on the int8 grid.
+__device__ __forceinline__ float sym_r(float a) {
+  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+  return isinf(r) ? 0.0f : r;
+}
+
+// Its scale S = a/127, 0 where sym_r gave 0 for a finite a.
+__device__ __forceinline__ float sym_S(float a, float r) {
+  return r > 0.0f || isinf(a) ? __fdiv_rn(a, 127.0f) : 0.0f;
+}
+
 // The low bytes of four words, a in the lowest byte (two byte permutes).
 __device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
@@ -507,13 +520,23 @@ __device__ __forceinline__ void dequant16(const uint4 &v, float S, int z, float 
   }
 }
 
-// Running per-halfword maximum of bf16 magnitudes (two values per word).
-__device__ __forceinline__ uint32_t absmax2_u4(const uint4 &v, uint32_t m2) {
-  m2 = __vmaxu2(m2, v.x & 0x7FFF7FFFu);
-  m2 = __vmaxu2(m2, v.y & 0x7FFF7FFFu);
-  m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
-  m2 = __vmaxu2(m2, v.w & 0x7FFF7FFFu);
+// Running absmax of the bf16 pairs of v, one packed max of magnitudes per
+// word: each half of the result is max(|m2 half|, |v half|) with the sign bit
+// meaningless (it is the xor of the operands' signs), so clear the sign bits
+// (absmax2_halves) before reading it. A NaN operand gives the canonical NaN
+// 0x7FFF, above every finite or infinite magnitude.
+__device__ __forceinline__ uint32_t absmax2_bf16(const uint4 &v, uint32_t m2) {
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m2) : "r"(v.x));
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m2) : "r"(v.y));
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m2) : "r"(v.z));
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m2) : "r"(v.w));
   return m2;
+}
+
+// The larger magnitude of the two halves of a running absmax2_bf16 value.
+__device__ __forceinline__ uint32_t absmax2_halves(uint32_t m2) {
+  m2 &= 0x7FFF7FFFu;
+  return max(m2 & 0xFFFFu, m2 >> 16);
 }
 
 

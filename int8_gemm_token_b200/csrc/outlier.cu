@@ -211,6 +211,20 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
     }
   }
 
+  // this thread's chunks are the same columns in every row: their outlier
+  // masks (one bit per column, one byte per chunk), gathered once
+  uint32_t mk[(VPT + 3) / 4];
+  uint32_t mk_any = 0;
+#pragma unroll
+  for (int i = 0; i < (VPT + 3) / 4; ++i) mk[i] = 0;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int64_t c = t + static_cast<int64_t>(j) * G;
+    if (G > 32 && c < chunks) mk[j >> 2] |= ((s_bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu) << ((j & 3) * 8);
+  }
+#pragma unroll
+  for (int i = 0; i < (VPT + 3) / 4; ++i) mk_any |= mk[i];
+
   for (int it = 0; grp < groups; grp += gridDim.x, ++it) {
     const int64_t m = grp * R + g;
     const bool row_ok = m < M;
@@ -226,13 +240,12 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
     const bool next_ok = grp + gridDim.x < groups && mn < M;
     uint4 nxt[kPrefetch ? VPT : 1];
     if constexpr (kPrefetch) load_row_chunks<G, VPT>(X + mn * ldx, chunks, t, next_ok, nxt);
-    uint32_t amax = 0;
+    if (G <= 32 || mk_any) {  // zero the outlier columns of this thread's chunks
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      const int64_t c = t + static_cast<int64_t>(j) * G;
-      if (row_ok && c < chunks) {
-        // zero the outlier columns of this 8-column chunk
-        const uint32_t mask8 = (s_bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu;
+      for (int j = 0; j < VPT; ++j) {
+        const int64_t c = t + static_cast<int64_t>(j) * G;
+        const uint32_t mask8 = G > 32 ? (mk[j >> 2] >> ((j & 3) * 8)) & 0xFFu
+                                      : (c < chunks ? (s_bits[c >> 2] >> ((c & 3) * 8)) & 0xFFu : 0u);
         if (mask8) {
           uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
@@ -242,10 +255,15 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
           }
           v[j] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        amax = absmax2_u4(v[j], amax);
       }
     }
-    amax = max(amax & 0xFFFFu, amax >> 16);
+    uint32_t amax = 0;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int64_t c = t + static_cast<int64_t>(j) * G;
+      if (row_ok && c < chunks) amax = absmax2_bf16(v[j], amax);
+    }
+    amax = absmax2_halves(amax);
     amax = __reduce_max_sync(0xFFFFFFFFu, amax);
     if (G > 32) {  // one row per block: combine the warps (double-buffered, one barrier per row)
       if ((tid & 31) == 0) red[it & 1][tid >> 5] = amax;
@@ -256,8 +274,8 @@ __global__ void __launch_bounds__(256) outlier_row_kernel(const uint16_t *__rest
     }
     if (row_ok) {
       const float a = __uint_as_float(amax << 16);
-      const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
-      if (t == 0) S_x[m] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+      const float r = sym_r(a);
+      if (t == 0) S_x[m] = sym_S(a, r);
       int8_t *qrow = Xq + m * K;
 #pragma unroll
       for (int j = 0; j < VPT; ++j) {

@@ -55,12 +55,12 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__
     const int64_t c = t + static_cast<int64_t>(j) * G;
     if (row_ok && c < chunks) {
       v[j] = __ldcs(reinterpret_cast<const uint4 *>(xrow) + c);
-      m2 = absmax2_u4(v[j], m2);
+      m2 = absmax2_bf16(v[j], m2);
     } else {
       v[j] = make_uint4(0, 0, 0, 0);
     }
   }
-  uint32_t amax = max(m2 & 0xFFFFu, m2 >> 16);
+  uint32_t amax = absmax2_halves(m2);
   amax = __reduce_max_sync(0xFFFFFFFFu, amax);
   if (G > 32) {
     if ((tid & 31) == 0) red[tid >> 5] = amax;
@@ -71,9 +71,8 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint16_t *__
   }
   if (!row_ok) return;
   const float a = __uint_as_float(amax << 16);
-  float r = 0.0f;
-  if (a > 0.0f) r = __fdiv_rn(127.0f, a);
-  if (t == 0) S_x[m] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+  const float r = sym_r(a);
+  if (t == 0) S_x[m] = sym_S(a, r);
   int8_t *qrow = Xq + m * K;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
@@ -295,19 +294,20 @@ __global__ void __launch_bounds__(256) calibrate_minmax_kernel(const T *__restri
 }
 
 // Pass 2 (one thread): S = (hi - lo)/255, r = 255/(hi - lo),
-// Z = clamp(-128 - rne(lo * r), -128, 127); all-zero data gives S = r = 1, Z = 0.
+// Z = clamp(-128 - rne(lo * r), -128, 127); all-zero data, or a range so
+// small that 255/(hi - lo) overflows fp32, gives S = r = 1, Z = 0.
 __global__ void calibrate_finalize_kernel(float *S, float *r, int32_t *Z) {
   const float hi = __uint_as_float(*reinterpret_cast<uint32_t *>(S));
   const float nlo = __uint_as_float(*reinterpret_cast<uint32_t *>(r));
   const float lo = nlo > 0.0f ? -nlo : 0.0f;
-  if (hi == lo) {
+  const float d = __fsub_rn(hi, lo);
+  const float rr = __fdiv_rn(255.0f, d);
+  if (hi == lo || isinf(rr)) {
     *S = 1.0f;
     *r = 1.0f;
     *Z = 0;
     return;
   }
-  const float d = __fsub_rn(hi, lo);
-  const float rr = __fdiv_rn(255.0f, d);
   *S = __fdiv_rn(d, 255.0f);
   *r = rr;
   *Z = min(max(-128 - rne_clamped(__fmul_rn(lo, rr)), -128), 127);
@@ -361,8 +361,8 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const T *__restrict__
   a = red[0][tx];
 #pragma unroll
   for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w][tx]);
-  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
-  if (ty == 0 && col_ok) s_w[n] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+  const float r = sym_r(a);
+  if (ty == 0 && col_ok) s_w[n] = sym_S(a, r);
 
   int32_t cs = 0;
   const int wr = threadIdx.x >> 3;  // output row (channel) this thread writes, 0..31

@@ -50,6 +50,21 @@ def check_split(X, threshold, cap, ld_pad=0):
     return rn, st
 
 
+@pytest.mark.parametrize("M,K", [(40, 4096), (300, 8192), (12, 2048)])
+def test_split_tiny_rows(M, K):
+    """Rows whose masked absmax is below 127/FLT_MAX (tiny values everywhere
+    but in the outlier columns) quantize as zero rows, as in the oracle."""
+    rng = np.random.default_rng(M + K)
+    Xf = np.clip(rng.standard_normal((M, K), dtype=np.float32), -5.5, 5.5)
+    tiny = np.array([1e-38, -1e-38, 3e-39, -9.2e-41, 0.0, -0.0, 2e-40, -5e-39], np.float32)
+    Xf[2:6] = rng.choice(tiny, size=(4, K))
+    cols = [3, K // 2 + 1, K - 1]
+    Xf[:, cols] = 20.0
+    X = synth.bf16_bits(Xf)
+    n, st = check_split(X, 6.0, 16)
+    assert n == len(cols) and st == 0
+
+
 @pytest.mark.parametrize("M,K,cols,ld_pad", [
     (3, 16, [2, 9], 0), (16, 256, [7, 100, 255], 8), (300, 4112, [0, 33, 4095, 4111], 0),
     (129, 1024, [], 0), (2, 65536, [5, 65535], 0), (4096, 8192, [11, 512, 777, 4000, 6001, 8191], 0),

@@ -55,6 +55,52 @@ def test_quant_per_token_ties():
     assert list(host(Xq)[0, :8]) == [127, 0, 0, 2, 2, -2, 4, 4]
 
 
+TINY = np.array([1e-38, -1e-38, 3e-39, -9.2e-41, 0.0, -0.0, 2e-40, -5e-39], np.float32)
+EDGE = np.array([4e-37, -4e-37, 1e-37, 0.0, -3e-38, 2e-39], np.float32)
+
+
+@pytest.mark.parametrize("M,K", [(6, 48), (6, 4096), (40, 11008), (300, 8192)])
+def test_quant_per_token_tiny_rows(M, K):
+    """Rows whose absmax is below 127/FLT_MAX (bf16 subnormals and tiny
+    normals) between ordinary rows quantize as zero rows (127/a overflows
+    fp32); a row just above that bound has a finite scale. Bit for bit as in
+    the oracle."""
+    rng = np.random.default_rng(K + 1)
+    X = synth.activations(rng, M, K)
+    X[1:4] = synth.bf16_bits(rng.choice(TINY, size=(3, K)))
+    X[4] = synth.bf16_bits(rng.choice(EDGE, size=K))
+    X[M - 1] = synth.bf16_bits(rng.choice(TINY[4:], size=K))
+    Xq, S = W.w8a8_quant_per_token(dev_bf16(X))
+    rq, rS = oracle.quant_per_token(X)
+    assert np.all(rq[1:4] == 0) and np.all(rS[1:4] == 0) and rS[4] > 0
+    assert_same(host(Xq), rq, "Xq")
+    assert_same(host(S), rS, "S_x")
+
+
+def test_calibrate_tiny_range():
+    """A calibration range whose 255/d overflows fp32 counts as empty
+    (S = r = 1, Z = 0); one just above it has a finite r."""
+    for Xf in (np.resize(TINY, (4, 64)), np.resize(EDGE * 4, (4, 64))):
+        X = synth.bf16_bits(Xf)
+        S, r, Z = W.w8a8_calibrate_static(dev_bf16(X))
+        rS, rr, rZ = oracle.calibrate_static(X)
+        assert host(S)[0] == rS and host(r)[0] == rr and host(Z)[0] == rZ
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_weight_quant_tiny_columns(dtype):
+    rng = np.random.default_rng(3)
+    Wf = synth.weight(rng, 256, 40)
+    Wf[:, 5:9] = rng.choice(TINY, size=(256, 4))
+    Wf[:, 11] = rng.choice(EDGE, size=256)
+    Wh = synth.bf16_bits(Wf) if dtype == "bf16" else Wf
+    Wq, s_w, cs = W.w8a8_quant_weight_per_channel(dev_bf16(Wh) if dtype == "bf16" else dev(Wh))
+    rq, rs, rc = oracle.quant_weight_per_channel(Wh)
+    assert_same(host(Wq), rq, "Wq")
+    assert_same(host(s_w), rs, "s_w")
+    assert_same(host(cs), rc, "colsum")
+
+
 @pytest.mark.parametrize("M,K", [(1, 4096), (32, 4096), (4096, 4096), (5, 48)])
 def test_calibrate_and_quant_per_tensor_bit_exact(M, K):
     case = synth.decode_static(M=min(M, 64), N=16, K=K, seed=M)
