@@ -442,13 +442,29 @@ __device__ __forceinline__ uint32_t pack_sat_s8x4(int a, int b, int c, int d) {
 
 // Symmetric codes of the 8 bf16 values in one uint4: clamp(rne(x * r), -127, 127). With r = 127/absmax every |x * r|
 // is at most 127 * (1 + 2^-23), so saturating to [-128, 127] equals that clamp.
+// The two fp32 products x0 * r and x1 * r, each rounded to nearest even, in
+// one packed fp32x2 multiply. Only for products that are rounded on their own:
+// ptxas contracts a packed multiply followed by a packed add into a fused
+// multiply-add, so no packed add may take these products.
+__device__ __forceinline__ void mul_f32x2(float x0, float x1, float r, float &p0, float &p1) {
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\t"
+      "mov.b64 pb, {%4, %4};\n\t"
+      "mul.rn.f32x2 pd, pa, pb;\n\t"
+      "mov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(p0), "=f"(p1)
+      : "f"(x0), "f"(x1), "f"(r));
+}
+
 __device__ __forceinline__ uint2 quant8_sym_sat(const uint4 &v, float r) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   int q[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    q[2 * i] = rne_s32(__fmul_rn(bf16_lo(w[i]), r));
-    q[2 * i + 1] = rne_s32(__fmul_rn(bf16_hi(w[i]), r));
+    float p0, p1;
+    mul_f32x2(bf16_lo(w[i]), bf16_hi(w[i]), r, p0, p1);
+    q[2 * i] = rne_s32(p0);
+    q[2 * i + 1] = rne_s32(p1);
   }
   return make_uint2(pack_sat_s8x4(q[0], q[1], q[2], q[3]), pack_sat_s8x4(q[4], q[5], q[6], q[7]));
 }
