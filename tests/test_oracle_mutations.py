@@ -43,6 +43,8 @@ MUTATIONS = {
     "bf16_round_half_away": ("u += 0x7fffu + keep_lsb;", "u += 0x8000u;"),
     "dequant_zero_point_added": ("float y = S * (float)((int32_t)Xq[m * K + k] - Z);",
                                  "float y = S * (float)((int32_t)Xq[m * K + k] + Z);"),
+    "tiny_vector_scale_overflow_unchecked": ("if (a > 0.0f && 127.0f / a <= FLT_MAX) {", "if (a > 0.0f) {"),
+    "tiny_range_calibration_unchecked": ("if (hi == lo || !(255.0f / d <= FLT_MAX)) {", "if (hi == lo) {"),
     "weight_read_along_rows": ("absmax_quant_vector(W, dtype, n, ldw, K, NULL, Wq + n * K, 1, &s_w[n]);",
                                "absmax_quant_vector(W, dtype, n, 1, K, NULL, Wq + n * K, 1, &s_w[n]);"),
 }
