@@ -169,6 +169,8 @@ def test_gemm_int32_accumulator_bit_exact(M, N, K):
 @pytest.mark.parametrize("M,N,K", [(16, 512, 256), (300, 520, 400), (200, 264, 512), (520, 5000, 400),
                                    (520, 5400, 256), (520, 5800, 272), (200, 11008, 512), (100, 2000, 400),
                                    (2048, 20480, 512), (1000, 18000, 208),
+                                   # the dispatch edges: Decode kernel up to 64 rows, 1-CTA up to 255, pair from 256
+                                   (64, 1000, 512), (65, 1000, 512), (255, 520, 400), (256, 520, 400),
                                    # CTA-pair tiles: rows of bf16 output that are not 16-byte multiples
                                    # (direct stores), and one tile whose only valid 64-column box is partial
                                    (260, 1001, 272), (300, 40, 128)])
