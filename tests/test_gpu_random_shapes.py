@@ -6,8 +6,9 @@ kernels; these draw their sizes instead: the Prefill linear (per-token
 quantization, then the INT8 GEMM with its dequant epilogue) for 1 to 600 rows,
 which spans the Decode-shaped, the 1-CTA and the CTA-pair kernels; the Decode
 linear with static quantization for 1 to 64 rows (the one-kernel and the
-two-kernel forms); and the LLM.int8() split followed by the CUDA-core mixed
-GEMM with 0 to 20 outlier columns.
+two-kernel forms); the LLM.int8() split followed by the CUDA-core mixed GEMM
+with 0 to 20 outlier columns; and the tensor-core side product with 0 to 100,
+held to its derived per-element bound.
 """
 import numpy as np
 import pytest
@@ -98,3 +99,39 @@ def test_llm_int8_random_shape(seed):
     rwq, rws, _ = oracle.quant_weight_per_channel(Wb)
     *_, y = oracle.linear_mixed(X, Wb, rwq, rws, threshold=6.0, cap=cap, bias=bias)
     assert_same(host_bf16(out), oracle.f32_to_bf16(y), f"out {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_llm_int8_tensor_core_side_random_shape(seed):
+    """The tensor-core side product at random shapes and outlier counts (0 to
+    100 columns, any cap above them), held to the same per-element bound as
+    its hand-picked cases (the fp32 side sums differ from the oracle's only
+    in their order)."""
+    from tests.test_gpu_outlier import side_tolerance
+
+    rng, M, N, K = draw(300 + seed, 600, 1500, 2048)
+    n_cols = int(rng.integers(0, min(100, K) + 1))
+    cap = n_cols + int(rng.integers(0, 40)) if n_cols else int(rng.integers(1, 40))
+    cols = np.sort(rng.choice(K, size=n_cols, replace=False))
+    x = np.clip(rng.standard_normal((M, K)).astype(np.float32), -5.5, 5.5)
+    x[:, cols] = (np.where(rng.random((M, n_cols)) < 0.5, -1.0, 1.0) * rng.uniform(20, 100, (M, n_cols))).astype(np.float32)
+    X = synth.bf16_bits(x)
+    Wb = synth.bf16_bits(synth.weight(rng, K, N))
+    bias = synth.bias(rng, N) if rng.random() < 0.5 else None
+    Wd = dev_bf16(Wb)
+    Wq, s_w, _ = W.w8a8_quant_weight_per_channel(Wd)
+    Xq, S_x, idx, n_out, Xo = W.int8_outlier_split(dev_bf16(X), 6.0, cap)
+    y32 = W.int8_mixed_decomp_gemm_tc(Xq, S_x, Xo, idx, n_out, cap, Wq, s_w, Wd,
+                                      bias=None if bias is None else dev(bias), out_dtype=torch.float32)
+    rq, rS, ridx, rn, rXo = oracle.outlier_split(X, 6.0, cap)
+    assert rn == n_cols and int(host(n_out)[0]) == rn
+    rwq, rws, _ = oracle.quant_weight_per_channel(Wb)
+    side = oracle.outlier_side(rXo, ridx, Wb)
+    y_ref = oracle.epilogue(oracle.gemm_i64(rq, rwq), rS, rws, bias=bias, side=side)
+    got = host(y32)
+    if n_cols == 0:
+        assert_same(got, y_ref, f"out {M}x{N}x{K}")
+        return
+    tol, _ = side_tolerance(rXo, ridx, Wb, side, bias, y_ref)
+    err = np.abs(got.astype(np.float64) - y_ref.astype(np.float64))
+    assert (err <= tol).all(), f"{M}x{N}x{K}, {n_cols} columns: {int((err > tol).sum())} elements outside the bound"
