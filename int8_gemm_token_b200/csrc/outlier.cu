@@ -21,14 +21,17 @@
 //   them cost about 3 us per call).
 // Pass 2 (rows): a grid sized to fill the SMs once; every CTA turns the
 //   bitmap into the ascending index list (block-wide popcount scan) and
-//   copies the bitmap into shared memory once; CTA 0 publishes the list and
-//   the count. The CTA then walks rows with a grid stride: each row is
-//   loaded once into registers (16-byte loads), with the next row's loads in
-//   flight when two rows fit in registers, outlier columns are masked to zero, the absmax is reduced with
-//   warp shuffles, the row is quantized from registers, and the row's
-//   outlier values are gathered into Xo. Pass 2 is launched with
-//   programmatic dependent launch and issues its first row loads before it
-//   waits for pass 1 (X is not written by pass 1).
+//   copies the bitmap into shared memory once, and each thread takes from it
+//   the masks of its own columns (the same in every row); CTA 0 publishes
+//   the list and the count. The CTA then walks rows with a grid stride: each
+//   row is loaded once into registers (16-byte loads), with the next row's
+//   loads in flight when two rows fit in registers; the row's first outlier
+//   value per thread is requested at the top of the row, outlier columns are
+//   masked to zero, the absmax is reduced (packed bf16 maxima, then warp
+//   shuffles), the row is quantized from registers, and the row's outlier
+//   values are stored into Xo. Pass 2 is launched with programmatic
+//   dependent launch and issues its first row loads before it waits for
+//   pass 1 (X is not written by pass 1).
 #include "device.cuh"
 #include "kernels.h"
 
