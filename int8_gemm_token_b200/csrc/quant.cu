@@ -3,8 +3,9 @@
 //  * quant_per_token:  PDMIX glossary §2.3 eq. Q_prefill with Z_token = 0
 //    (configuration guide: Prefill is per-token symmetric); LLM.int8()
 //    summary §一.1 absmax equation. One fused pass: 16-byte loads of the row
-//    into registers, absmax by warp shuffles, one fp32 division per row,
-//    quantize from registers, 8-byte int8 stores.
+//    into registers, absmax by packed bf16 maxima and warp shuffles, one fp32
+//    division per row (a row whose 127/absmax overflows fp32 is quantized as
+//    zero), quantize from registers, 8-byte int8 stores.
 //  * quant_per_tensor: PDMIX glossary §2.3 eq. Q_decode (static S, Z).
 //  * dequant_per_tensor: its inverse x = S (q - Z), the read side of an INT8
 //    KV cache kept in the Decode scheme.
@@ -17,9 +18,6 @@
 
 namespace w8a8 {
 
-// ------------------------------------------------------------------ helpers
-// |x| of bf16 values compared on their bit patterns: for finite values the
-// magnitude bits order exactly like the magnitudes.
 // ------------------------------------------------------------ per token
 // G threads per row (32 = one warp, or 256 = the whole block), VPT 16-byte
 // chunks (8 bf16) per thread held in registers, so X is read exactly once.
